@@ -1,0 +1,298 @@
+"""Plain fp64 CPU oracle of the top-k routed MoE FFN forward pass.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
+CPU-baseline leg of bench.py, never by the product path. It shares no code with
+the CUDA library; the only thing both sides share is the seeded input
+generator module, which holds none of the layer's arithmetic.
+
+Every function follows the pages step by step, with numpy fp64 matrix products
+as the only library primitive. Sources (page title, then section):
+
+  [ZTF]  Zero to Frontier, ch. 13 section 13.1 "Why MoE": "The MoE layer"
+         (router r = x W_r, TopK, gate softmax over the kept logits, SwiGLU
+         experts, MoE(x) = sum_{i in K} g_i FFN_i(x)); "Total and active
+         parameters"; "Mixtral 8x7B, counted exactly"; "DeepSeek-V3, counted
+         exactly"; "In PyTorch" (loop over experts; FLOP table).
+  [KL]   kevinluzbetak "Mixture-Of-Experts": routing paragraph (p =
+         softmax(h W_r), keep top-k, renormalise), balancing list
+         (E * sum_i f_i P_i) and the capacity worked example.
+  [AEI]  AI Engineering Illustrated, "Mixture of Experts": "The router is
+         small but it decides everything" (router in float32), "The safety
+         valve is a capacity limit" (dropped tokens skip the expert),
+         "Fine-grained experts and a shared expert".
+  [JP]   jacopoparretti "Mixture of experts, token by token": "A hard limit"
+         (capacity), "A penalty" (Switch balance statistic).
+
+Readings taken where the pages are silent or disagree (each listed in the
+design notes):
+  R1 top-k ties go to the lower expert index;
+  R2 the router logit is the exact dot product rounded once to float32
+     (the pages fix the router precision at float32); every later step is fp64;
+  R3 capacity C = floor(cf * T * k / E); within an expert the first C
+     assignments in token order are kept; gates are not renormalised over the
+     survivors; a dropped assignment contributes 0;
+  R4 f_i = routed assignments to i / (T k), counted before the capacity cut;
+     P_i = mean over tokens of the full softmax; the statistic is E sum f_i P_i
+     with no alpha weight;
+  R5 the shared expert is added with weight 1 and is never dropped;
+  R6 an optional per-expert router bias is added to the logits before both the
+     softmax and the top-k.
+The drop ordering of R3 is "parity unpinned" by the pages: it is fixed only by
+this definition and a hand-built case.
+"""
+from __future__ import annotations
+
+import math
+from typing import Callable, Optional, Sequence
+
+import numpy as np
+
+__all__ = [
+    "router_logits", "softmax_all", "top_k", "gates_softmax_topk", "gates_renormalised",
+    "topk_margin", "capacity_limit", "capacity_keep", "silu", "swiglu_ffn",
+    "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
+    "moe_param_count", "active_flops", "OracleResult",
+]
+
+
+def _f64(a) -> np.ndarray:
+    """Exact upcast of a numpy array or a (CPU) torch tensor to float64."""
+    if hasattr(a, "detach"):  # torch tensor: bf16 -> fp32 is exact, then fp64
+        a = a.detach().to("cpu").float().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Router  ([ZTF] "The MoE layer"; [AEI] router precision; [KL] routing paragraph)
+# ----------------------------------------------------------------------------
+
+def router_logits(x, W_r, bias=None) -> np.ndarray:
+    """Router logits r = x W_r for every token, one per expert.
+
+    x: [T, d]; W_r: [E, d] (the router matrix stored expert-major, i.e. W_r^T of
+    the page's d x E map); bias: optional [E] added to every token's logits (R6).
+    The sum is taken in fp64 on the exact input values, then rounded once to
+    float32 (R2); the result is returned as float64 holding float32 values.
+    """
+    r = _f64(x) @ _f64(W_r).T
+    if bias is not None:
+        r = r + _f64(bias)[None, :]
+    return r.astype(np.float32).astype(np.float64)
+
+
+def softmax_all(r: np.ndarray) -> np.ndarray:
+    """p = softmax(r) over all E experts, per token, max-subtracted ([KL])."""
+    z = r - r.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def top_k(r: np.ndarray, k: int) -> np.ndarray:
+    """The set K = TopK(r, k) per token, as indices [T, k] in slot order.
+
+    Slot order is descending logit; equal logits go to the lower index (R1).
+    A stable sort of -r keeps equal keys in index order, which is that rule.
+    """
+    order = np.argsort(-r, axis=1, kind="stable")
+    return order[:, :k].astype(np.int64)
+
+
+def gates_softmax_topk(r: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """g_i = e^{r_i} / sum_{j in K} e^{r_j} for i in K ([ZTF] "The MoE layer")."""
+    rk = np.take_along_axis(r, idx, axis=1)
+    z = np.exp(rk - rk.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def gates_renormalised(p: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """g = p_K / sum(p_K): softmax over all experts, keep the top-k, renormalise ([KL])."""
+    pk = np.take_along_axis(p, idx, axis=1)
+    return pk / pk.sum(axis=1, keepdims=True)
+
+
+def topk_margin(r: np.ndarray, k: int) -> np.ndarray:
+    """Gap between the k-th and (k+1)-th largest logit per token (+inf when k = E).
+
+    Where this gap is tiny, either top-k set is a correct answer for logits
+    carrying float32 rounding, so comparisons of routing decisions use it.
+    """
+    E = r.shape[1]
+    if k >= E:
+        return np.full(r.shape[0], np.inf)
+    s = -np.sort(-r, axis=1)
+    return s[:, k - 1] - s[:, k]
+
+
+# ----------------------------------------------------------------------------
+# Capacity  ([AEI] "The safety valve is a capacity limit"; [JP] "A hard limit";
+#            [KL] capacity worked example)
+# ----------------------------------------------------------------------------
+
+def capacity_limit(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
+    """Per-expert slot limit C = floor(cf * T * k / E) (R3); None when cf <= 0."""
+    if capacity_factor is None or capacity_factor <= 0:
+        return None
+    return int(math.floor(float(capacity_factor) * T * k / E))
+
+
+def capacity_keep(idx: np.ndarray, E: int, C: Optional[int]) -> np.ndarray:
+    """Keep mask [T, k]: per expert, the first C assignments in token order (R3)."""
+    T, k = idx.shape
+    keep = np.ones((T, k), dtype=bool)
+    if C is None:
+        return keep
+    seen = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for s in range(k):
+            e = idx[t, s]
+            keep[t, s] = seen[e] < C
+            seen[e] += 1
+    return keep
+
+
+def dropped_fraction(counts: np.ndarray, C: Optional[int], T: int, k: int) -> float:
+    """Share of the T*k assignments that overflow their expert's capacity."""
+    if C is None:
+        return 0.0
+    return float(np.maximum(0, np.asarray(counts) - C).sum()) / (T * k)
+
+
+# ----------------------------------------------------------------------------
+# Experts  ([ZTF] "The MoE layer": FFN_i(x) = (SiLU(x W_g) (.) x W_u) W_d)
+# ----------------------------------------------------------------------------
+
+def silu(a: np.ndarray) -> np.ndarray:
+    """SiLU(a) = a * sigmoid(a) = a / (1 + e^{-a})."""
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-a))
+
+
+def swiglu_ffn(x, W_g, W_u, W_d) -> np.ndarray:
+    """One SwiGLU expert on rows x [n, d].
+
+    W_g, W_u: [d_e, d] and W_d: [d, d_e] in nn.Linear weight layout, so the
+    page's x W_g is x @ W_g.T here.
+    """
+    x = _f64(x)
+    a = x @ _f64(W_g).T
+    b = x @ _f64(W_u).T
+    return (silu(a) * b) @ _f64(W_d).T
+
+
+# ----------------------------------------------------------------------------
+# Balance statistic  ([KL] balancing list; [JP] "A penalty";
+#                     [AEI] "Fix 1 adds an auxiliary loss")
+# ----------------------------------------------------------------------------
+
+def aux_statistic(counts: np.ndarray, probsum: np.ndarray, T: int, k: int) -> float:
+    """E * sum_i f_i P_i with f_i = counts_i / (T k) and P_i = probsum_i / T (R4)."""
+    E = len(counts)
+    f = np.asarray(counts, dtype=np.float64) / (T * k)
+    P = np.asarray(probsum, dtype=np.float64) / T
+    return float(E * np.sum(f * P))
+
+
+def aux_statistic_top1(idx: np.ndarray, p: np.ndarray) -> float:
+    """Variant in which f counts only each token's first choice (for reference)."""
+    T, E = p.shape
+    f = np.bincount(idx[:, 0], minlength=E) / T
+    return float(E * np.sum(f * p.mean(axis=0)))
+
+
+# ----------------------------------------------------------------------------
+# The layer
+# ----------------------------------------------------------------------------
+
+class OracleResult:
+    """Everything the oracle computes for one layer call."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
+                capacity_factor: float = 0.0, router_bias=None,
+                shared_weights: Optional[Sequence] = None,
+                rows: Optional[np.ndarray] = None) -> OracleResult:
+    """Forward pass of the routed MoE FFN layer, looping over experts.
+
+    x: [T, d]; W_r: [E, d]; expert_weights(e) -> (W_g[e], W_u[e], W_d[e]);
+    shared_weights: (gate [d_s,d], up [d_s,d], down [d,d_s]) or None.
+    rows: the token indices whose output y is evaluated (default: all). Routing,
+    counts, capacity and the balance statistic always cover all T tokens.
+
+    Steps ([KL] routing paragraph and layer listing; [ZTF] "The MoE layer" and
+    "In PyTorch"): logits for every token; softmax over all experts; top-k;
+    gates; counts; capacity cut in token order; then for each expert, its kept
+    tokens in one batch through the SwiGLU, scaled by the gate and added into y;
+    the shared expert on every token with weight 1; the balance statistic.
+    """
+    T = x.shape[0]
+    r = router_logits(x, W_r, router_bias)
+    E = r.shape[1]
+    p = softmax_all(r)
+    idx = top_k(r, k)
+    g = gates_softmax_topk(r, idx)
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.int64)
+    C = capacity_limit(capacity_factor, T, k, E)
+    keep = capacity_keep(idx, E, C)
+    probsum = p.sum(axis=0)
+    aux = aux_statistic(counts, probsum, T, k)
+
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    want = np.zeros(T, dtype=bool)
+    want[rows] = True
+    xr = _f64(x) if not hasattr(x, "detach") else None  # lazy: convert rows only
+    d = x.shape[1]
+    y = np.zeros((T, d), dtype=np.float64)
+    for e in range(E):
+        tok, slot = np.nonzero((idx == e) & keep & want[:, None])
+        if tok.size == 0:
+            continue
+        Wg, Wu, Wd = expert_weights(e)
+        xe = xr[tok] if xr is not None else _f64(x[tok])
+        y[tok] += g[tok, slot][:, None] * swiglu_ffn(xe, Wg, Wu, Wd)
+    if shared_weights is not None:
+        xs = xr[rows] if xr is not None else _f64(x[rows])
+        y[rows] += swiglu_ffn(xs, *shared_weights)
+
+    return OracleResult(logits=r, probs=p, idx=idx, gates=g, counts=counts,
+                        capacity=C, keep=keep, probsum=probsum, aux=aux,
+                        margin=topk_margin(r, k), rows=rows, y=y[rows],
+                        dropped_fraction=dropped_fraction(counts, C, T, k))
+
+
+# ----------------------------------------------------------------------------
+# Parameter and FLOP accounting ([ZTF] "Total and active parameters",
+# "Mixtral 8x7B, counted exactly", "DeepSeek-V3, counted exactly", "FLOPs per
+# token, and the 6N rule for MoE" and the dense-versus-MoE table)
+# ----------------------------------------------------------------------------
+
+def moe_param_count(cfg: dict) -> tuple:
+    """(total, active) parameters of a decoder with MoE FFN layers.
+
+    cfg keys: V, d, L, attn (attention parameters per layer), n_dense (leading
+    layers with a dense FFN of width d_ff), d_ff, E (routed experts), E_shared,
+    k, d_e, tied. Every FFN/expert is a bias-free SwiGLU (3 d width matrices),
+    each layer has two RMSNorm gains of size d, there is one final norm, the
+    router is a bias-free d x E matrix, and embeddings count in full in both.
+    """
+    d = cfg["d"]
+    norms = 2 * d
+    expert = 3 * d * cfg["d_e"]
+    router = d * cfg["E"]
+    dense_layer = cfg["attn"] + norms + 3 * d * cfg.get("d_ff", 0)
+    moe_total = cfg["attn"] + norms + (cfg["E"] + cfg.get("E_shared", 0)) * expert + router
+    moe_active = cfg["attn"] + norms + (cfg["k"] + cfg.get("E_shared", 0)) * expert + router
+    n_dense = cfg.get("n_dense", 0)
+    n_moe = cfg["L"] - n_dense
+    emb = cfg["V"] * d * (1 if cfg.get("tied", False) else 2)
+    total = n_dense * dense_layer + n_moe * moe_total + emb + d
+    active = n_dense * dense_layer + n_moe * moe_active + emb + d
+    return total, active
+
+
+def active_flops(kept_assignments: int, d: int, d_e: int, T: int = 0, d_s: int = 0) -> int:
+    """Forward FLOPs of the expert products: 2 per multiply-add, 3 d d_e per
+    assignment, plus the shared expert's 3 d d_s per token (router excluded)."""
+    return 2 * 3 * d * d_e * int(kept_assignments) + 2 * 3 * d * d_s * int(T)
