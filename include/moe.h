@@ -1,0 +1,173 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of a top-k routed
+ * mixture-of-experts SwiGLU FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (Zero to Frontier, ch. 13 section 13.1 "Why MoE",
+ * "The MoE layer"; kevinluzbetak "Mixture-Of-Experts", routing paragraph):
+ *
+ *   r   = x W_r (+ b)                    router logits, one per expert, fp32
+ *   p   = softmax(r)                     over all E experts
+ *   K   = TopK(r, k)                     ties go to the lower expert index
+ *   g_i = e^{r_i} / sum_{j in K} e^{r_j} (the same as p_K / sum p_K)
+ *   y   = sum_{i in K, kept} g_i FFN_i(x) + FFN_shared(x)
+ *   FFN(x) = (SiLU(x W_g) * (x W_u)) W_d
+ *   aux = E * sum_i f_i P_i              f_i = routed assignments / (T k),
+ *                                        P_i = mean_t p_ti
+ *
+ * Capacity (AI Engineering Illustrated "Mixture of Experts", "The safety valve
+ * is a capacity limit"; jacopoparretti "Mixture of experts, token by token",
+ * "A hard limit"; kevinluzbetak capacity example): when capacity_factor > 0,
+ * each expert keeps at most C = floor(capacity_factor * T * k / E)
+ * assignments, the first C in token order; a dropped assignment contributes
+ * 0 (the token keeps its other experts' terms, gates are not renormalised).
+ * The shared expert is never dropped and has weight 1.
+ *
+ * The Switch balance statistic (kevinluzbetak balancing list; jacopoparretti
+ * "A penalty") is returned raw, without the trainer's alpha weight.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is owned by the caller. Device pointers are CUDA device
+ *     memory of the current device; host pointers are ordinary (ideally
+ *     pinned) host memory. The library allocates no memory.
+ *   - Arrays are row-major and dense. Device pointers must be 16-byte aligned.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and return MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE.
+ *   - moe_forward is asynchronous on dims->stream; a CUDA launch failure
+ *     returns MOE_ERR_CUDA. Bounded device-side waits record a timeout that
+ *     moe_get_device_status reports after the caller synchronises.
+ *   - Calls on one stream are ordered; two calls that share one workspace
+ *     must not overlap on the device.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, NaN factor */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid layer this build does not run (see limits below) */
+  MOE_ERR_WORKSPACE = 3,      /* workspace null, too small or misaligned */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a device-side bounded wait gave up (moe_get_device_status) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Number of kernels moe_forward enqueues, in order: router logits, routing
+ * (softmax / top-k / gates / ranks), scan (counts, capacity, offsets, aux),
+ * scatter (permute x rows), gate/up grouped GEMM + SwiGLU, down grouped GEMM
+ * + gate scaling, combine (un-permute + shared expert). */
+#define MOE_NUM_KERNELS 7
+
+/* Limits of this build: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
+ * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1). */
+
+typedef struct {
+  int64_t T;                 /* tokens in this call (0 allowed: empty batch) */
+  int32_t d;                 /* model width */
+  int32_t d_e;               /* routed expert hidden width */
+  int32_t d_s;               /* shared expert hidden width; 0 = no shared expert */
+  int32_t dtype;             /* moe_dtype of x, W_g, W_u, W_d, W_shared and y */
+  int32_t gate_mode;         /* 0 = renormalised top-k gates (only value accepted) */
+  const float* router_bias;  /* device [E] fp32 added to the logits before softmax
+                                and top-k, or NULL */
+  void* workspace;           /* device scratch of >= moe_workspace_size() bytes,
+                                256-byte aligned, owned by the caller */
+  size_t workspace_bytes;
+  void* stream;              /* cudaStream_t to enqueue on; NULL = default stream */
+  void* const* events;       /* optional cudaEvent_t[2*MOE_NUM_KERNELS]; when non-NULL,
+                                events[2i] / events[2i+1] are recorded on `stream`
+                                right before / after kernel i (NULL entries skipped) */
+} moe_dims;
+
+/* Bytes of device workspace moe_forward needs for this layer (0 on invalid
+ * arguments). Depends on T, d, d_e, d_s, dtype, E, k and capacity_factor. */
+MOE_API size_t moe_workspace_size(const moe_dims* dims, int E, int k, float capacity_factor);
+
+/* Capacity C = floor(capacity_factor * T * k / E) the forward pass applies,
+ * or -1 when capacity_factor <= 0 (no limit). */
+MOE_API int64_t moe_capacity(int64_t T, int E, int k, float capacity_factor);
+
+/*
+ * Forward pass of the routed MoE FFN layer (see top of file).
+ *   x        device [T, d]            dtype
+ *   W_r      device [E, d]            fp32 (the router's d x E matrix, stored expert-major)
+ *   W_g, W_u device [E, d_e, d]       dtype (nn.Linear weight layout: K contiguous)
+ *   W_d      device [E, d, d_e]       dtype
+ *   W_shared device, packed [gate (d_s x d) | up (d_s x d) | down (d x d_s)], or
+ *            NULL when dims->d_s == 0
+ *   y        device [T, d]            dtype, written (every row)
+ *   aux      device float[1]          written: E * sum_i f_i P_i (0 when T == 0)
+ *   counts   device int32[E]          written: routed assignments per expert,
+ *                                     before the capacity cut
+ * Enqueues MOE_NUM_KERNELS kernels on dims->stream, no host synchronisation.
+ */
+MOE_API moe_status moe_forward(const moe_dims* dims,
+                       const void* x, const float* W_r, const void* W_g,
+                       const void* W_u, const void* W_d, const void* W_shared,
+                       int E, int k, float capacity_factor,
+                       void* y, float* aux, int32_t* counts);
+
+/*
+ * End-to-end variant for callers holding the activations in host memory: the
+ * same forward pass, bracketed by the copies. Copies x_host -> x_dev, runs
+ * moe_forward, copies y_dev -> y_host, aux_dev -> aux_host and counts_dev ->
+ * counts_host, all on dims->stream, then synchronises that stream and returns
+ * moe_get_device_status() if the pass itself succeeded. Weights stay device
+ * pointers. x_host / y_host should be pinned for full copy bandwidth.
+ */
+MOE_API moe_status moe_forward_host_io(const moe_dims* dims,
+                               const void* x_host, void* x_dev,
+                               const float* W_r, const void* W_g, const void* W_u,
+                               const void* W_d, const void* W_shared,
+                               int E, int k, float capacity_factor,
+                               void* y_dev, void* y_host,
+                               float* aux_dev, float* aux_host,
+                               int32_t* counts_dev, int32_t* counts_host);
+
+/* Where moe_forward keeps its routing results inside the workspace (byte
+ * offsets from dims->workspace), so that callers and tests can read them after
+ * the call. Valid until the next call that uses the same workspace. */
+typedef struct {
+  size_t logits;      /* fp32 [T, E]    router logits x W_r (bias not included) */
+  size_t topk_idx;    /* int32 [T, k]   chosen experts, descending logit */
+  size_t gates;       /* fp32 [T, k]    gates of those experts */
+  size_t slot_pos;    /* int32 [T, k]   row of each assignment in the permuted
+                                        buffers, or -1 when dropped */
+  size_t probsum;     /* fp64 [E]       sum over tokens of the full softmax */
+  size_t tile_start;  /* int32 [E + 1]  first 128-row tile of each expert's
+                                        segment; [E] = number of routed tiles */
+  size_t xp;          /* dtype [rows_max, d]   x rows grouped by expert */
+  size_t h;           /* dtype [rows_max, d_e] SwiGLU hidden rows */
+  size_t yrows;       /* dtype [rows_max, d]   gate-scaled expert outputs */
+  int64_t rows_max;   /* rows reserved for the permuted buffers */
+  int64_t capacity;   /* C, or -1 */
+} moe_workspace_layout_t;
+
+MOE_API moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capacity_factor,
+                                moe_workspace_layout_t* out);
+
+/* Status of the device-side bounded waits since the last call (for the current
+ * device); resets it. Call after synchronising the stream(s) used.
+ * MOE_OK or MOE_ERR_DEVICE_TIMEOUT (or MOE_ERR_CUDA if it cannot be read). */
+MOE_API moe_status moe_get_device_status(void);
+
+/* Static, human-readable name of a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

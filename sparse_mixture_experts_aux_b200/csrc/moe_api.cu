@@ -1,0 +1,501 @@
+// libmoe.so: C ABI of the routed MoE FFN forward pass (include/moe.h).
+// Host side: argument checks, workspace layout, TMA descriptors and the launch
+// sequence; the kernels live in the included headers (one translation unit).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "moe.h"
+#include "common.cuh"
+#include "router.cuh"
+#include "permute.cuh"
+#include "tc_gemm.cuh"
+
+namespace {
+
+using moe::ROW_TILE;
+
+constexpr size_t ALIGN = 1024;
+constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s per mbarrier wait
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Plan {
+  int64_t T;
+  int d, de, ds, E, k;
+  bool bf16;
+  size_t esz;
+  int64_t C;  // -1: no limit
+  int nblk;   // routing chunks
+  int64_t rows_max;
+  size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
+      o_tile_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys, total;
+};
+
+int64_t capacity_of(int64_t T, int E, int k, float cf) {
+  if (!(cf > 0.f)) return -1;  // <= 0 (NaN is rejected earlier): no limit
+  const double c = floor(static_cast<double>(cf) * static_cast<double>(T) * k / E);
+  const double cap = static_cast<double>(T) * k;
+  return c >= cap ? static_cast<int64_t>(cap) : static_cast<int64_t>(c);
+}
+
+moe_status check_dims(const moe_dims* dims, int E, int k, float cf) {
+  if (dims == nullptr) return MOE_ERR_INVALID_ARG;
+  if (dims->T < 0 || dims->d <= 0 || dims->d_e <= 0 || dims->d_s < 0) return MOE_ERR_INVALID_ARG;
+  if (dims->dtype != MOE_F32 && dims->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (isnan(cf)) return MOE_ERR_INVALID_ARG;
+  if (dims->gate_mode != 0) return MOE_ERR_UNSUPPORTED;
+  if (E > moe::tc::MAX_E || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (dims->T * static_cast<int64_t>(k) >= (int64_t(1) << 31) ||
+      dims->T * static_cast<int64_t>(E) >= (int64_t(1) << 40))
+    return MOE_ERR_UNSUPPORTED;
+  const int mult = dims->dtype == MOE_BF16 ? 64 : 32;
+  if (dims->d % mult || dims->d_e % mult || dims->d_s % mult) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
+  Plan p{};
+  p.T = dims->T;
+  p.d = dims->d;
+  p.de = dims->d_e;
+  p.ds = dims->d_s;
+  p.E = E;
+  p.k = k;
+  p.bf16 = dims->dtype == MOE_BF16;
+  p.esz = p.bf16 ? 2 : 4;
+  p.C = capacity_of(p.T, E, k, cf);
+  p.nblk = static_cast<int>((p.T + moe::ROUTE_CHUNK - 1) / moe::ROUTE_CHUNK);
+  p.rows_max = static_cast<int64_t>(
+      align_up(static_cast<size_t>(p.T * k + static_cast<int64_t>(ROW_TILE - 1) * E), ROW_TILE));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, ALIGN);
+    return o;
+  };
+  const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
+  p.o_logits = take(T * E * 4);
+  p.o_idx = take(TK * 4);
+  p.o_gate = take(TK * 4);
+  p.o_lrank = take(TK * 4);
+  p.o_slot = take(TK * 4);
+  p.o_hist = take(static_cast<size_t>(p.nblk) * E * 4);
+  p.o_base = take(static_cast<size_t>(p.nblk) * E * 4);
+  p.o_psum_part = take(static_cast<size_t>(p.nblk) * moe::ROUTE_WARPS * E * 8);
+  p.o_probsum = take(static_cast<size_t>(E) * 8);
+  p.o_tile_start = take(static_cast<size_t>(E + 1) * 4);
+  p.o_rowgate = take(R * 4);
+  p.o_xp = take(R * p.d * p.esz);
+  p.o_h = take(R * p.de * p.esz);
+  p.o_yrows = take(R * p.d * p.esz);
+  p.o_hs = take(p.ds ? T * p.ds * p.esz : 0);
+  p.o_ys = take(p.ds ? T * p.d * p.esz : 0);
+  p.total = off;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// Per-device one-time set-up: SM count and kernel attributes.
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+moe_status device_setup(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.ready) {
+    if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return MOE_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    const int smem = moe::tc::SMEM_BYTES;
+    if (cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int rs = 2 * moe::ROUTE_WARPS * moe::tc::MAX_E * 4;
+    if (cudaFuncSetAttribute(moe::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             rs) != cudaSuccess ||
+        cudaFuncSetAttribute(moe::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             rs) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    di.ready = true;
+  }
+  *num_sms = di.num_sms;
+  return MOE_OK;
+}
+
+// bf16 tensor map over a row-major [outer][mid][inner] array (mid = 1 for 2D),
+// 128-byte swizzle, box {64, box_rows(, 1)}; out-of-range rows read as zero.
+bool encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                uint32_t box_rows, int rank) {
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::tc::BK), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct Timer {
+  void* const* ev;
+  cudaStream_t s;
+  void at(int i) const {
+    if (ev != nullptr && ev[i] != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
+  }
+};
+
+moe_status launched() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename TX>
+moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const TX* x,
+                                    const float* W_r, uint8_t* ws, int32_t* counts, float* aux,
+                                    cudaStream_t st, const Timer& tm) {
+  float* logits = reinterpret_cast<float*>(ws + P.o_logits);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + P.o_idx);
+  float* gate = reinterpret_cast<float*>(ws + P.o_gate);
+  int32_t* lrank = reinterpret_cast<int32_t*>(ws + P.o_lrank);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + P.o_slot);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + P.o_hist);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + P.o_base);
+  double* psum_part = reinterpret_cast<double*>(ws + P.o_psum_part);
+  double* probsum = reinterpret_cast<double*>(ws + P.o_probsum);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(ws + P.o_tile_start);
+  float* rowgate = reinterpret_cast<float*>(ws + P.o_rowgate);
+  TX* xp = reinterpret_cast<TX*>(ws + P.o_xp);
+  const int T = static_cast<int>(P.T);
+
+  // (0) router logits, fp32 FMA
+  moe::SimtGroup rg{};
+  rg.A = x;
+  rg.B0 = W_r;
+  rg.B1 = nullptr;
+  rg.b_stride = 0;
+  rg.C = logits;
+  rg.tile_start = nullptr;
+  rg.E = 1;
+  rg.rows = P.T;
+  rg.N = P.E;
+  rg.K = P.d;
+  rg.active = 1;
+  moe::SimtGroup none{};
+  tm.at(0);
+  {
+    dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM, 1);
+    moe::simt_gemm_kernel<TX, float, float, moe::EPI_STORE_F32><<<grid, 256, 0, st>>>(rg, none);
+  }
+  tm.at(1);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+
+  // (1) routing
+  tm.at(2);
+  {
+    const size_t smem = static_cast<size_t>(2) * moe::ROUTE_WARPS * P.E * 4;
+    const int nv = (P.E + 31) / 32;
+#define MOE_ROUTE(NV)                                                                           \
+  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(logits, dims->router_bias, T, P.E, P.k, idx, \
+                                                   gate, lrank, hist, psum_part)
+    if (nv <= 1) MOE_ROUTE(1);
+    else if (nv <= 2) MOE_ROUTE(2);
+    else if (nv <= 4) MOE_ROUTE(4);
+    else if (nv <= 8) MOE_ROUTE(8);
+    else if (nv <= 16) MOE_ROUTE(16);
+    else MOE_ROUTE(32);
+#undef MOE_ROUTE
+  }
+  tm.at(3);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+
+  // (2) scan: counts, capacity, segment offsets, aux
+  tm.at(4);
+  moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk * moe::ROUTE_WARPS, P.E,
+                                       P.T, P.k, P.C, counts, base, tile_start, probsum, aux);
+  tm.at(5);
+  if (launched() != MOE_OK) return MOE_ERR_CUDA;
+
+  // (3) scatter rows into expert segments
+  tm.at(6);
+  moe::scatter_kernel<TX><<<(T + 7) / 8, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
+                                                       base, tile_start, slot, rowgate, xp);
+  tm.at(7);
+  return launched();
+}
+
+moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, const void* W_g,
+                        const void* W_u, const void* W_d, const void* W_shared, int E, int k,
+                        float cf, void* y, float* aux, int32_t* counts) {
+  moe_status s = check_dims(dims, E, k, cf);
+  if (s != MOE_OK) return s;
+  if (aux == nullptr || counts == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(aux, 4) || !aligned(counts, 4)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(dims->stream);
+  if (dims->T == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess ||
+        cudaMemsetAsync(aux, 0, sizeof(float), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (x == nullptr || W_r == nullptr || W_g == nullptr || W_u == nullptr || W_d == nullptr ||
+      y == nullptr || (dims->d_s > 0 && W_shared == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_r, W_g, W_u, W_d, y};
+  for (const void* q : ptrs)
+    if (!aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  if (dims->d_s > 0 && !aligned(W_shared, 16)) return MOE_ERR_INVALID_ARG;
+  if (dims->router_bias != nullptr && !aligned(dims->router_bias, 16)) return MOE_ERR_INVALID_ARG;
+
+  const Plan P = make_plan(dims, E, k, cf);
+  if (dims->workspace == nullptr || !aligned(dims->workspace, 256) ||
+      dims->workspace_bytes < P.total)
+    return MOE_ERR_WORKSPACE;
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != MOE_OK) return s;
+
+  uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
+  const Timer tm{dims->events, st};
+  const int T = static_cast<int>(P.T);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + P.o_slot);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(ws + P.o_tile_start);
+  float* rowgate = reinterpret_cast<float*>(ws + P.o_rowgate);
+
+  if (P.bf16) {
+    using bf16 = __nv_bfloat16;
+    s = launch_route_and_permute<bf16>(P, dims, static_cast<const bf16*>(x), W_r, ws, counts, aux,
+                                       st, tm);
+    if (s != MOE_OK) return s;
+    const bf16* xp = reinterpret_cast<const bf16*>(ws + P.o_xp);
+    bf16* h = reinterpret_cast<bf16*>(ws + P.o_h);
+    bf16* yrows = reinterpret_cast<bf16*>(ws + P.o_yrows);
+    bf16* hs = P.ds ? reinterpret_cast<bf16*>(ws + P.o_hs) : nullptr;
+    bf16* ys = P.ds ? reinterpret_cast<bf16*>(ws + P.o_ys) : nullptr;
+    const bf16* sg = static_cast<const bf16*>(W_shared);
+    const size_t sh_n = static_cast<size_t>(P.ds) * P.d;
+    const int ng = P.ds ? 2 : 1;
+
+    // (4) gate/up projection + SwiGLU
+    {
+      moe::tc::TcMaps maps;
+      memset(&maps, 0, sizeof(maps));
+      bool ok = encode_map(&maps.a[0], xp, P.d, P.rows_max, 1, moe::tc::BM, 2) &&
+                encode_map(&maps.b0[0], W_g, P.d, P.de, E, moe::tc::BN / 2, 3) &&
+                encode_map(&maps.b1[0], W_u, P.d, P.de, E, moe::tc::BN / 2, 3);
+      if (P.ds)
+        ok = ok && encode_map(&maps.a[1], x, P.d, P.T, 1, moe::tc::BM, 2) &&
+             encode_map(&maps.b0[1], sg, P.d, P.ds, 1, moe::tc::BN / 2, 3) &&
+             encode_map(&maps.b1[1], sg + sh_n, P.d, P.ds, 1, moe::tc::BN / 2, 3);
+      if (!ok) return MOE_ERR_CUDA;
+      moe::tc::TcParams tp{};
+      tp.num_groups = ng;
+      tp.timeout_ns = kWaitTimeoutNs;
+      tp.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                 P.d / moe::tc::BK, P.de, h, nullptr};
+      if (P.ds)
+        tp.g[1] = {nullptr, 1, T, (P.ds + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                   P.d / moe::tc::BK, P.ds, hs, nullptr};
+      tm.at(8);
+      moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>
+          <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(maps, tp);
+      tm.at(9);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    }
+    // (5) down projection, scaled by the assignment's gate
+    {
+      moe::tc::TcMaps maps;
+      memset(&maps, 0, sizeof(maps));
+      bool ok = encode_map(&maps.a[0], h, P.de, P.rows_max, 1, moe::tc::BM, 2) &&
+                encode_map(&maps.b0[0], W_d, P.de, P.d, E, moe::tc::BN, 3);
+      if (P.ds)
+        ok = ok && encode_map(&maps.a[1], hs, P.ds, P.T, 1, moe::tc::BM, 2) &&
+             encode_map(&maps.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, moe::tc::BN, 3);
+      if (!ok) return MOE_ERR_CUDA;
+      maps.b1[0] = maps.b0[0];
+      maps.b1[1] = maps.b0[1];
+      moe::tc::TcParams tp{};
+      tp.num_groups = ng;
+      tp.timeout_ns = kWaitTimeoutNs;
+      tp.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
+                 P.d, yrows, rowgate};
+      if (P.ds)
+        tp.g[1] = {nullptr, 1, T, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.ds / moe::tc::BK, P.d,
+                   ys, nullptr};
+      tm.at(10);
+      moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>
+          <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(maps, tp);
+      tm.at(11);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    }
+    // (6) combine
+    tm.at(12);
+    moe::combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+                                                           static_cast<bf16*>(y));
+    tm.at(13);
+    return launched();
+  }
+
+  // fp32 layer: the same pipeline with fp32 FMA expert products
+  const float* xf = static_cast<const float*>(x);
+  s = launch_route_and_permute<float>(P, dims, xf, W_r, ws, counts, aux, st, tm);
+  if (s != MOE_OK) return s;
+  const float* xp = reinterpret_cast<const float*>(ws + P.o_xp);
+  float* h = reinterpret_cast<float*>(ws + P.o_h);
+  float* yrows = reinterpret_cast<float*>(ws + P.o_yrows);
+  float* hs = P.ds ? reinterpret_cast<float*>(ws + P.o_hs) : nullptr;
+  float* ys = P.ds ? reinterpret_cast<float*>(ws + P.o_ys) : nullptr;
+  const float* sg = static_cast<const float*>(W_shared);
+  const size_t sh_n = static_cast<size_t>(P.ds) * P.d;
+  const int64_t gy = (P.rows_max > P.T ? P.rows_max : P.T);
+  {
+    moe::SimtGroup a{}, b{};
+    a = {xp, W_g, W_u, static_cast<int64_t>(P.de) * P.d, h, nullptr, tile_start, E, 0, P.de, P.d,
+         1};
+    if (P.ds) b = {xf, sg, sg + sh_n, 0, hs, nullptr, nullptr, 1, P.T, P.ds, P.d, 1};
+    const int nmax = P.de > P.ds ? P.de : P.ds;
+    dim3 grid((nmax + moe::SG_BN - 1) / moe::SG_BN,
+              static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
+    tm.at(8);
+    moe::simt_gemm_kernel<float, float, float, moe::EPI_SWIGLU><<<grid, 256, 0, st>>>(a, b);
+    tm.at(9);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  }
+  {
+    moe::SimtGroup a{}, b{};
+    a = {h, W_d, nullptr, static_cast<int64_t>(P.d) * P.de, yrows, rowgate, tile_start, E, 0, P.d,
+         P.de, 1};
+    if (P.ds) b = {hs, sg + 2 * sh_n, nullptr, 0, ys, nullptr, nullptr, 1, P.T, P.d, P.ds, 1};
+    dim3 grid((P.d + moe::SG_BN - 1) / moe::SG_BN,
+              static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
+    tm.at(10);
+    moe::simt_gemm_kernel<float, float, float, moe::EPI_SCALE><<<grid, 256, 0, st>>>(a, b);
+    tm.at(11);
+    if (launched() != MOE_OK) return MOE_ERR_CUDA;
+  }
+  tm.at(12);
+  moe::combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+                                                          static_cast<float*>(y));
+  tm.at(13);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims* dims, int E, int k, float capacity_factor) {
+  if (check_dims(dims, E, k, capacity_factor) != MOE_OK) return 0;
+  return make_plan(dims, E, k, capacity_factor).total;
+}
+
+int64_t moe_capacity(int64_t T, int E, int k, float capacity_factor) {
+  if (T < 0 || E < 1 || k < 1) return -1;
+  return capacity_of(T, E, k, capacity_factor);
+}
+
+moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capacity_factor,
+                                moe_workspace_layout_t* out) {
+  const moe_status s = check_dims(dims, E, k, capacity_factor);
+  if (s != MOE_OK) return s;
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  const Plan P = make_plan(dims, E, k, capacity_factor);
+  out->logits = P.o_logits;
+  out->topk_idx = P.o_idx;
+  out->gates = P.o_gate;
+  out->slot_pos = P.o_slot;
+  out->probsum = P.o_probsum;
+  out->tile_start = P.o_tile_start;
+  out->xp = P.o_xp;
+  out->h = P.o_h;
+  out->yrows = P.o_yrows;
+  out->rows_max = P.rows_max;
+  out->capacity = P.C;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_dims* dims, const void* x, const float* W_r, const void* W_g,
+                       const void* W_u, const void* W_d, const void* W_shared, int E, int k,
+                       float capacity_factor, void* y, float* aux, int32_t* counts) {
+  return forward_impl(dims, x, W_r, W_g, W_u, W_d, W_shared, E, k, capacity_factor, y, aux,
+                      counts);
+}
+
+moe_status moe_get_device_status(void) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, moe::g_dev_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(moe::g_dev_error, &zero, sizeof(int)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_forward_host_io(const moe_dims* dims, const void* x_host, void* x_dev,
+                               const float* W_r, const void* W_g, const void* W_u, const void* W_d,
+                               const void* W_shared, int E, int k, float capacity_factor,
+                               void* y_dev, void* y_host, float* aux_dev, float* aux_host,
+                               int32_t* counts_dev, int32_t* counts_host) {
+  moe_status s = check_dims(dims, E, k, capacity_factor);
+  if (s != MOE_OK) return s;
+  if (aux_host == nullptr || counts_host == nullptr) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (x_host == nullptr || y_host == nullptr)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(dims->stream);
+  const size_t esz = dims->dtype == MOE_BF16 ? 2 : 4;
+  const size_t bytes = static_cast<size_t>(dims->T) * dims->d * esz;
+  if (bytes && cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  s = forward_impl(dims, x_dev, W_r, W_g, W_u, W_d, W_shared, E, k, capacity_factor, y_dev,
+                   aux_dev, counts_dev);
+  if (s != MOE_OK) return s;
+  if ((bytes && cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
+      cudaMemcpyAsync(aux_host, aux_dev, sizeof(float), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(counts_host, counts_dev, sizeof(int32_t) * E, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  return moe_get_device_status();
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_STATUS_UNKNOWN";
+}
+
+}  // extern "C"

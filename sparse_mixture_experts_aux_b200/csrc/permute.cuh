@@ -1,0 +1,91 @@
+// Permute (scatter of token rows into expert-grouped segments, with the
+// capacity cut) and combine (gate-weighted un-permute plus the shared expert).
+//
+// Sources: Zero to Frontier 13.1 "Why MoE", "In PyTorch" (gather each
+// expert's tokens into one batch, add the weighted result back; a sort by
+// expert replaces the loop's bookkeeping); kevinluzbetak "Mixture-Of-Experts"
+// (production layers sort tokens by expert; capacity example: overflow
+// assignments skip the expert, the token keeps its other expert's term);
+// AI Engineering Illustrated "Mixture of Experts", "The safety valve is a
+// capacity limit".
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// One warp per token. Lane s (< k) resolves assignment s: its rank in token
+// order within the expert is base[chunk][e] + lrank; it is kept when the rank
+// is below the capacity C, and lands at row tile_start[e]*ROW_TILE + rank.
+// The token's row is then copied to every kept position with 16-byte loads
+// and stores (coalesced across the warp).
+template <typename TX>
+__global__ void __launch_bounds__(256) scatter_kernel(
+    const TX* __restrict__ x, int d, int T, int k, int E, int64_t C,
+    const int32_t* __restrict__ idx, const float* __restrict__ gate,
+    const int32_t* __restrict__ lrank, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ tile_start, int32_t* __restrict__ slot_pos,
+    float* __restrict__ row_gate, TX* __restrict__ xp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;  // warp-uniform
+  int mypos = -1;
+  if (lane < k) {
+    const size_t a = (size_t)t * k + lane;
+    const int e = idx[a];
+    const int rank = base[(size_t)(t / ROUTE_CHUNK) * E + e] + lrank[a];
+    if (C < 0 || (int64_t)rank < C) {
+      mypos = tile_start[e] * ROW_TILE + rank;
+      row_gate[mypos] = gate[a];
+    }
+    slot_pos[a] = mypos;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  const int nvec = (int)((size_t)d * sizeof(TX) / 16);
+  for (int s = 0; s < k; ++s) {
+    const int p = __shfl_sync(0xffffffffu, mypos, s);
+    if (p < 0) continue;
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)p * d);
+    for (int c = lane; c < nvec; c += 32) st_v4(dst + c, ld_nc_v4(src + c));
+  }
+}
+
+// One warp per token: y[t] = sum_s Yrows[slot_pos[t][s]] (dropped slots skipped)
+// + Ys[t] (shared expert, if any), summed in fp32 in slot order with a single
+// rounding to the output type. Yrows already carry the gate factor.
+template <typename TY>
+__global__ void __launch_bounds__(256) combine_kernel(
+    const TY* __restrict__ yrows, const TY* __restrict__ ys, const int32_t* __restrict__ slot_pos,
+    int T, int k, int d, TY* __restrict__ y) {
+  constexpr int VN = Vec16<TY>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;  // warp-uniform
+  const int mypos = (lane < k) ? slot_pos[(size_t)t * k + lane] : -1;
+  const int nvec = (int)((size_t)d * sizeof(TY) / 16);
+  for (int c0 = 0; c0 < nvec; c0 += 32) {
+    const int c = c0 + lane;
+    const bool active = c < nvec;
+    float acc[VN];
+#pragma unroll
+    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+    for (int s = 0; s < k; ++s) {
+      const int p = __shfl_sync(0xffffffffu, mypos, s);
+      if (p >= 0 && active) {
+        float f[VN];
+        Vec16<TY>::unpack(ld_v4(reinterpret_cast<const uint4*>(yrows + (size_t)p * d) + c), f);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] += f[i];
+      }
+    }
+    if (!active) continue;
+    if (ys != nullptr) {
+      float f[VN];
+      Vec16<TY>::unpack(ld_v4(reinterpret_cast<const uint4*>(ys + (size_t)t * d) + c), f);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[i] += f[i];
+    }
+    st_v4(reinterpret_cast<uint4*>(y + (size_t)t * d) + c, Vec16<TY>::pack(acc));
+  }
+}
+
+}  // namespace moe

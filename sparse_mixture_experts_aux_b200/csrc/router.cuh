@@ -1,0 +1,364 @@
+// Router logits, routing (softmax / top-k / gates / stable ranks) and the scan
+// that turns per-chunk expert histograms into counts, capacity cuts, padded
+// segment offsets and the Switch balance statistic.
+//
+// Sources: Zero to Frontier 13.1 "Why MoE", "The MoE layer" (r = x W_r, TopK,
+// gates = softmax over the kept logits); kevinluzbetak "Mixture-Of-Experts",
+// routing paragraph (softmax over all, top-k, renormalise) and balancing list
+// (E * sum_i f_i P_i); AI Engineering Illustrated "Mixture of Experts", "The
+// router is small but it decides everything" (router in float32) and "The
+// safety valve is a capacity limit".
+#pragma once
+#include "common.cuh"
+#include <math.h>
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// SIMT fp32 "TN" GEMM: C[m, n] = sum_k A[m, k] * B[e][n, k], both operands
+// K-contiguous, fp32 FMA accumulation (no TF32). Used for the router logits
+// (A = x, B = W_r) and for the fp32 layer's expert products, where the
+// rows of A are grouped per expert in ROW_TILE-padded segments.
+// ---------------------------------------------------------------------------
+enum { EPI_STORE_F32 = 0, EPI_SWIGLU = 1, EPI_SCALE = 2 };
+
+struct SimtGroup {
+  const void* A;            // [rows, K]
+  const void* B0;           // expert e at B0 + e * b_stride  ([N, K] each)
+  const void* B1;           // second operand of the SwiGLU (up projection)
+  int64_t b_stride;         // elements between experts
+  void* C;                  // [rows, N]
+  const float* row_scale;   // EPI_SCALE: multiplier per row (NULL = 1)
+  const int32_t* tile_start;// grouped rows: [E + 1] segment starts in ROW_TILE units; NULL = dense
+  int E;
+  int64_t rows;             // dense: number of valid rows
+  int N, K;
+  int active;               // 0: this grid z-slice does nothing
+};
+
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+
+template <typename TA>
+__device__ __forceinline__ void load4(const TA* p, float* f);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, float* f) {
+  float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v.x));
+  float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v.y));
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+template <typename TA, typename TB, typename TC, int EPI>
+__global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup g1) {
+  const SimtGroup g = blockIdx.z == 0 ? g0 : g1;
+  if (!g.active) return;
+  const int n0 = blockIdx.x * SG_BN;
+  const int64_t m0 = (int64_t)blockIdx.y * SG_BM;
+  if (n0 >= g.N) return;
+  int e = 0;
+  int64_t m_end;
+  if (g.tile_start) {
+    const int64_t total = (int64_t)g.tile_start[g.E] * ROW_TILE;
+    if (m0 >= total) return;
+    int lo = 0, hi = g.E - 1;  // last expert whose segment starts at or before m0
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)g.tile_start[mid] * ROW_TILE <= m0) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    m_end = (int64_t)g.tile_start[e + 1] * ROW_TILE;
+  } else {
+    if (m0 >= g.rows) return;
+    m_end = g.rows;
+  }
+  constexpr int NB = (EPI == EPI_SWIGLU) ? 2 : 1;
+  __shared__ float As[SG_BK][SG_BM + 4];
+  __shared__ float Bs[NB][SG_BK][SG_BN + 4];
+
+  const int tid = threadIdx.x;
+  const int lr = tid >> 2, lk = (tid & 3) * 4;
+  const int ty = tid >> 4, tx = tid & 15;
+  const TA* A = reinterpret_cast<const TA*>(g.A);
+  const TB* Bp[2] = {reinterpret_cast<const TB*>(g.B0) + (int64_t)e * g.b_stride,
+                     NB == 2 ? reinterpret_cast<const TB*>(g.B1) + (int64_t)e * g.b_stride : nullptr};
+  float acc[NB][4][4];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[b][i][j] = 0.f;
+
+  const int64_t arow = m0 + lr;
+  const int brow = n0 + lr;
+  for (int k0 = 0; k0 < g.K; k0 += SG_BK) {
+    float f[4] = {0.f, 0.f, 0.f, 0.f};
+    if (arow < m_end) load4<TA>(A + arow * g.K + k0 + lk, f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) As[lk + i][lr] = f[i];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float h[4] = {0.f, 0.f, 0.f, 0.f};
+      if (brow < g.N) load4<TB>(Bp[b] + (int64_t)brow * g.K + k0 + lk, h);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Bs[b][lk + i][lr] = h[i];
+    }
+    __syncthreads();
+    // Blocked summation: each K tile is summed into a fresh partial that is
+    // then added to the running total, which keeps the rounding error of a
+    // long dot product (d up to thousands) about sqrt(SG_BK) times smaller
+    // than one sequential chain.
+    float part[NB][4][4];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[b][i][j] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        float4 bq = *reinterpret_cast<const float4*>(&Bs[b][kk][tx * 4]);
+        float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[b][i][j] = fmaf(av[i], bv[j], part[b][i][j]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[b][i][j] += part[b][i][j];
+    __syncthreads();
+  }
+
+  TC* C = reinterpret_cast<TC*>(g.C);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t m = m0 + ty * 4 + i;
+    if (m >= m_end) continue;
+    float scale = 1.f;
+    if (EPI == EPI_SCALE && g.row_scale) scale = g.row_scale[m];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= g.N) continue;
+      float v;
+      if (EPI == EPI_SWIGLU) {
+        const float a = acc[0][i][j];
+        v = (a / (1.0f + expf(-a))) * acc[NB - 1][i][j];
+      } else if (EPI == EPI_SCALE) {
+        v = scale * acc[0][i][j];
+      } else {
+        v = acc[0][i][j];
+      }
+      C[m * g.N + n] = from_f32<TC>(v);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Routing: one warp per token, ROUTE_CHUNK tokens per block.
+//   softmax over all E logits (+ optional bias), per-expert probability sums
+//   accumulated in fp64 in a fixed order; top-k by k rounds of a warp argmax
+//   ordered by (logit descending, index ascending); gates as a softmax over
+//   the k kept logits; then stable ranks: for each assignment, how many
+//   earlier tokens of the same chunk chose the same expert (a 32-bit token
+//   mask per warp and expert, prefix-summed over the chunk's warps).
+// Outputs per block: hist[blk][e] and per-warp probability-sum partials.
+// NV = ceil(E / 32) logits held per lane.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int NV>
+__global__ void __launch_bounds__(256) route_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int32_t* __restrict__ lrank_out,
+    int32_t* __restrict__ hist, double* __restrict__ psum_part) {
+  extern __shared__ uint32_t route_smem[];
+  uint32_t* bm = route_smem;                                   // [ROUTE_WARPS][E] token masks
+  int32_t* wbase = reinterpret_cast<int32_t*>(route_smem + ROUTE_WARPS * E);  // [ROUTE_WARPS][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = blockIdx.x;
+  for (int i = threadIdx.x; i < ROUTE_WARPS * E; i += blockDim.x) bm[i] = 0u;
+  __syncthreads();
+
+  const int t_warp0 = blk * ROUTE_CHUNK + warp * 32;
+  double ps[NV];
+  float bv[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    ps[i] = 0.0;
+    const int e = lane + 32 * i;
+    bv[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+  }
+
+  for (int j = 0; j < 32; ++j) {
+    const int t = t_warp0 + j;
+    if (t >= T) break;  // warp-uniform
+    const float* row = logits + (size_t)t * E;
+    float v[NV];
+    uint32_t removed = 0u;
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        v[i] = row[e] + bv[i];
+        m = fmaxf(m, v[i]);
+      } else {
+        v[i] = -INFINITY;
+        removed |= 1u << i;
+      }
+    }
+    m = warp_max(m);
+    float ex[NV];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      ex[i] = (lane + 32 * i < E) ? expf(v[i] - m) : 0.f;
+      s += ex[i];
+    }
+    s = warp_sum(s);
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      if (lane + 32 * i < E) ps[i] += (double)(ex[i] / s);
+
+    int my_e = 0;
+    float my_v = 0.f;
+    for (int sl = 0; sl < k; ++sl) {
+      float best_v = -INFINITY;
+      int best_e = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        if (!((removed >> i) & 1u)) {
+          const int e = lane + 32 * i;
+          if (v[i] > best_v || (v[i] == best_v && e < best_e)) { best_v = v[i]; best_e = e; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
+        if (ov > best_v || (ov == best_v && oe < best_e)) { best_v = ov; best_e = oe; }
+      }
+      if (lane == sl) { my_e = best_e; my_v = best_v; }
+      if ((best_e & 31) == lane) removed |= 1u << (best_e >> 5);
+    }
+    const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+    const float z = (lane < k) ? expf(my_v - v0) : 0.f;
+    const float zs = warp_sum(z);
+    if (lane < k) {
+      idx_out[(size_t)t * k + lane] = my_e;
+      gate_out[(size_t)t * k + lane] = z / zs;
+    }
+  }
+  __syncwarp();
+
+  const int t = t_warp0 + lane;
+  if (t < T) {
+    for (int sl = 0; sl < k; ++sl) {
+      const int e = idx_out[(size_t)t * k + sl];
+      atomicOr(&bm[warp * E + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < ROUTE_WARPS; ++w) {
+      wbase[w * E + e] = run;
+      run += __popc(bm[w * E + e]);
+    }
+    hist[(size_t)blk * E + e] = run;
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) psum_part[((size_t)blk * ROUTE_WARPS + warp) * E + e] = ps[i];
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int sl = 0; sl < k; ++sl) {
+      const int e = idx_out[(size_t)t * k + sl];
+      lrank_out[(size_t)t * k + sl] = wbase[warp * E + e] + __popc(bm[warp * E + e] & lt);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Scan (one block of 1024 threads, thread e = expert e):
+//   base[b][e]   = assignments to e in chunks before b (stable token-order rank base)
+//   counts[e]    = routed assignments to e (before the capacity cut)
+//   kept_e       = min(counts[e], C); segment of ceil(kept_e / ROW_TILE) tiles
+//   tile_start   = exclusive scan of the segment sizes; tile_start[E] = total
+//   probsum[e]   = sum of the probability partials, fp64, fixed order
+//   aux          = E * sum_e (counts_e / (T k)) (probsum_e / T), fp64, fixed tree
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) scan_kernel(
+    const int32_t* __restrict__ hist, int nblk, const double* __restrict__ psum_part, int nparts,
+    int E, int64_t T, int k, int64_t C, int32_t* __restrict__ counts, int32_t* __restrict__ base,
+    int32_t* __restrict__ tile_start, double* __restrict__ probsum, float* __restrict__ aux) {
+  __shared__ int s_scan[2][1024];
+  __shared__ double s_sum[1024];
+  const int e = threadIdx.x;
+  int tiles = 0;
+  double term = 0.0;
+  if (e < E) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      base[(size_t)b * E + e] = run;
+      run += hist[(size_t)b * E + e];
+    }
+    counts[e] = run;
+    const int kept = (C >= 0 && (int64_t)run > C) ? (int)C : run;
+    tiles = (kept + ROW_TILE - 1) / ROW_TILE;
+    double ps = 0.0;
+    for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
+    probsum[e] = ps;
+    term = (double)run * ps;
+  }
+  s_scan[0][e] = tiles;
+  s_sum[e] = term;
+  __syncthreads();
+  int cur = 0;
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = s_scan[cur][e] + (e >= off ? s_scan[cur][e - off] : 0);
+    s_scan[cur ^ 1][e] = v;
+    cur ^= 1;
+    __syncthreads();
+  }
+  if (e < E) tile_start[e] = s_scan[cur][e] - tiles;
+  if (e == E - 1) tile_start[E] = s_scan[cur][e];
+  for (int half = 512; half > 0; half >>= 1) {  // fixed-shape tree sum
+    if (e < half) s_sum[e] += s_sum[e + half];
+    __syncthreads();
+  }
+  if (e == 0) {
+    const double denom = (double)T * (double)k * (double)T;
+    aux[0] = (T > 0) ? (float)((double)E * s_sum[0] / denom) : 0.f;
+  }
+}
+
+}  // namespace moe

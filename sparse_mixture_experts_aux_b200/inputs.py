@@ -58,6 +58,11 @@ MIXTRAL_DECODE = Workload("mixtral-decode T=32 d=4096 E=8 d_e=14336 k=2", 32, 40
 
 ALL_WORKLOADS = (TINY_F32, MIXTRAL, DEEPSEEK_V3, SWITCH_ZIPF, MIXTRAL_DECODE)
 
+# A smaller case with the Mixtral expert shape (about 1 GB on the device), for
+# hardware-counter captures of the same kernels.
+MIXTRAL_PROFILE = Workload("mixtral-shape-profile T=2048 d=4096 E=2 d_e=14336 k=2",
+                           2048, 4096, 2, 14336, 2, seed=1)
+
 
 def zipf_router_bias(E: int) -> torch.Tensor:
     """Per-expert logit offset log(1/rank^1.2) with rank = e + 1 (fp32)."""

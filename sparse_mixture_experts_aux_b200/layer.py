@@ -1,0 +1,100 @@
+"""Torch-facing wrapper of moe_forward: torch supplies device memory and the
+stream, the library does every step of the layer. Marshalling only."""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return _lib.MOE_BF16
+    if dt == torch.float32:
+        return _lib.MOE_F32
+    raise TypeError(f"unsupported activation dtype {dt}; expected bfloat16 or float32")
+
+
+class Workspace:
+    """A reusable device scratch buffer (torch-allocated, 512-byte aligned)."""
+
+    def __init__(self, device=None):
+        self.buf: Optional[torch.Tensor] = None
+        self.device = device
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, stream, events):
+    T, d = x.shape
+    d_e = W_g.shape[1]
+    return _lib.make_dims(T, d, d_e, d_s, dtype_code(x.dtype), router_bias, ws,
+                          ws.numel() if ws is not None else 0, stream, events)
+
+
+def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Tensor,
+            W_d: torch.Tensor, W_shared: Optional[torch.Tensor] = None, k: int = 2,
+            capacity_factor: float = 0.0, router_bias: Optional[torch.Tensor] = None,
+            d_s: int = 0, workspace: Optional[Workspace] = None, stream=None, events=None,
+            y: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
+            counts: Optional[torch.Tensor] = None):
+    """Run the routed MoE FFN layer; returns (y, aux[1] fp32, counts[E] int32) on x's device.
+
+    Shapes: x [T, d]; W_r [E, d] fp32; W_g, W_u [E, d_e, d]; W_d [E, d, d_e];
+    W_shared packed [gate d_s*d | up d_s*d | down d*d_s] when d_s > 0.
+    """
+    for name, t in (("x", x), ("W_r", W_r), ("W_g", W_g), ("W_u", W_u), ("W_d", W_d)):
+        if not t.is_cuda:
+            raise RuntimeError(f"{name} must be a CUDA tensor (the layer has no CPU path)")
+        if not t.is_contiguous():
+            raise RuntimeError(f"{name} must be contiguous")
+    E = W_r.shape[0]
+    dev = x.device
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    elif isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    workspace = workspace or Workspace()
+    probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events)
+    nbytes = _lib.moe_workspace_size(probe, E, k, capacity_factor)
+    if nbytes == 0:
+        raise _lib.MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    ws = workspace.get(nbytes, dev)
+    dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events)
+    y = torch.empty_like(x) if y is None else y
+    aux = torch.empty(1, dtype=torch.float32, device=dev) if aux is None else aux
+    counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
+    _lib.moe_forward(dims, x, W_r, W_g, W_u, W_d, W_shared, E, k, capacity_factor, y, aux, counts)
+    return y, aux, counts
+
+
+def routing_views(ws: torch.Tensor, x: torch.Tensor, W_g: torch.Tensor, E: int, k: int,
+                  capacity_factor: float = 0.0, d_s: int = 0) -> dict:
+    """Views of the routing results moe_forward left in workspace `ws`."""
+    T, d = x.shape
+    dims = _dims_for(x, W_g, d_s, None, ws, 0, None)
+    L = _lib.moe_workspace_layout(dims, E, k, capacity_factor)
+    b = ws
+
+    def view(off, n, dt):
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        return b[off:off + nbytes].view(dt)
+
+    d_e = W_g.shape[1]
+    return dict(
+        logits=view(L.logits, T * E, torch.float32).view(T, E),
+        topk_idx=view(L.topk_idx, T * k, torch.int32).view(T, k),
+        gates=view(L.gates, T * k, torch.float32).view(T, k),
+        slot_pos=view(L.slot_pos, T * k, torch.int32).view(T, k),
+        probsum=view(L.probsum, E, torch.float64),
+        tile_start=view(L.tile_start, E + 1, torch.int32),
+        xp=view(L.xp, L.rows_max * d, x.dtype).view(L.rows_max, d),
+        h=view(L.h, L.rows_max * d_e, x.dtype).view(L.rows_max, d_e),
+        yrows=view(L.yrows, L.rows_max * d, x.dtype).view(L.rows_max, d),
+        rows_max=L.rows_max, capacity=L.capacity,
+    )

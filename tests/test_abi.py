@@ -1,0 +1,157 @@
+"""The C ABI library loads, exports every symbol include/moe.h declares, and
+rejects bad arguments on the host before touching a GPU (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_mixture_experts_aux_b200 import _lib
+from sparse_mixture_experts_aux_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    hdr = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", hdr)
+
+
+def test_header_declares_the_binding_surface():
+    names = declared_symbols()
+    assert sorted(names) == sorted(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    # and nothing that is not declared is exported under the moe_ prefix
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(0) == "MOE_OK"
+    assert _lib.status_string(5) == "MOE_ERR_DEVICE_TIMEOUT"
+    assert _lib.status_string(99) == "MOE_STATUS_UNKNOWN"
+
+
+def test_capacity_matches_page_example(lib):
+    # kevinluzbetak capacity example: 4096 tokens, 4 experts, top-2, factor 1.25 -> 2560
+    assert _lib.moe_capacity(4096, 4, 2, 1.25) == 2560
+    assert _lib.moe_capacity(16384, 64, 1, 1.25) == 320
+    assert _lib.moe_capacity(100, 4, 2, 0.0) == -1
+    assert _lib.moe_capacity(100, 4, 2, -1.0) == -1
+    assert _lib.moe_capacity(8, 2, 1, 0.5) == 2
+    # a factor so large that no expert can overflow is clamped to T*k
+    assert _lib.moe_capacity(10, 2, 1, 1e30) == 10
+
+
+def test_capacity_agrees_with_oracle_formula(lib):
+    from oracle import moe_oracle as O
+    for T, E, k, cf in [(1000, 7, 3, 1.1), (333, 5, 2, 0.37), (4096, 64, 1, 2.0), (17, 3, 1, 0.99)]:
+        assert _lib.moe_capacity(T, E, k, cf) == O.capacity_limit(cf, T, k, E)
+
+
+def _dims(**kw):
+    base = dict(T=128, d=256, d_e=256, d_s=0, dtype=_lib.MOE_BF16)
+    base.update(kw)
+    return _lib.make_dims(**base)
+
+
+def test_workspace_size_and_layout(lib):
+    d = _dims()
+    n = _lib.moe_workspace_size(d, 8, 2, 0.0)
+    assert n > 0
+    L = _lib.moe_workspace_layout(d, 8, 2, 0.0)
+    # rows reserved cover T*k assignments plus per-expert padding to 128 rows
+    assert L.rows_max >= 128 * 2 + 127 * 8 and L.rows_max % 128 == 0
+    offs = [L.logits, L.topk_idx, L.gates, L.slot_pos, L.probsum, L.tile_start, L.xp, L.h, L.yrows]
+    assert all(o % 256 == 0 for o in offs)
+    assert max(offs) < n
+    assert L.capacity == -1
+    # a shared expert needs more scratch
+    assert _lib.moe_workspace_size(_dims(d_s=128), 8, 2, 0.0) > n
+
+
+@pytest.mark.parametrize("E,k,kw,want", [
+    (8, 0, {}, _lib.MOE_ERR_INVALID_ARG),          # k < 1
+    (8, 9, {}, _lib.MOE_ERR_INVALID_ARG),          # k > E
+    (0, 1, {}, _lib.MOE_ERR_INVALID_ARG),          # no experts
+    (2048, 2, {}, _lib.MOE_ERR_UNSUPPORTED),       # E above the build limit
+    (64, 33, {}, _lib.MOE_ERR_UNSUPPORTED),        # k above the build limit
+    (8, 2, dict(d=100), _lib.MOE_ERR_UNSUPPORTED),  # bf16 width not a multiple of 64
+    (8, 2, dict(d_e=96), _lib.MOE_ERR_UNSUPPORTED),
+    (8, 2, dict(d_s=32), _lib.MOE_ERR_UNSUPPORTED),
+    (8, 2, dict(dtype=_lib.MOE_F32, d=48), _lib.MOE_ERR_UNSUPPORTED),
+    (8, 2, dict(T=-1), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(d=0), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(dtype=7), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(gate_mode=1), _lib.MOE_ERR_UNSUPPORTED),
+])
+def test_forward_rejects_bad_shapes_on_host(lib, E, k, kw, want):
+    d = _dims(**kw)
+    st = _lib.moe_forward(d, 16, 16, 16, 16, 16, None, E, k, 0.0, 16, 16, 16, check=False)
+    assert st == want
+    assert _lib.moe_workspace_size(d, E, k, 0.0) == 0
+
+
+def test_forward_rejects_bad_pointers_on_host(lib):
+    d = _dims()
+    ws_bytes = _lib.moe_workspace_size(d, 8, 2, 0.0)
+    good = 1 << 20  # never dereferenced: every case below fails validation first
+    args = dict(x=good, W_r=good, W_g=good, W_u=good, W_d=good, W_shared=None, y=good, aux=good,
+                counts=good)
+
+    def call(dims=d, cf=0.0, **over):
+        a = dict(args, **over)
+        return _lib.moe_forward(dims, a["x"], a["W_r"], a["W_g"], a["W_u"], a["W_d"],
+                                a["W_shared"], 8, 2, cf, a["y"], a["aux"], a["counts"], check=False)
+
+    for name in ("x", "W_r", "W_g", "W_u", "W_d", "y", "aux", "counts"):
+        assert call(**{name: 0}) == _lib.MOE_ERR_INVALID_ARG, name
+    for name in ("x", "W_r", "W_g", "W_u", "W_d", "y"):
+        assert call(**{name: good + 8}) == _lib.MOE_ERR_INVALID_ARG, name  # misaligned
+    assert call(aux=good + 2) == _lib.MOE_ERR_INVALID_ARG
+    assert call(cf=float("nan")) == _lib.MOE_ERR_INVALID_ARG
+    # shared expert requested without its weights
+    assert call(dims=_dims(d_s=128)) == _lib.MOE_ERR_INVALID_ARG
+    # workspace missing, too small, misaligned
+    assert call() == _lib.MOE_ERR_WORKSPACE
+    small = _dims(workspace=good, workspace_bytes=ws_bytes - 1)
+    assert call(dims=small) == _lib.MOE_ERR_WORKSPACE
+    skew = _dims(workspace=good + 16, workspace_bytes=ws_bytes)
+    assert call(dims=skew) == _lib.MOE_ERR_WORKSPACE
+    assert _lib.moe_forward(None, good, good, good, good, good, None, 8, 2, 0.0, good, good, good,
+                            check=False) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from sparse_mixture_experts_aux_b200 import forward
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    w = torch.zeros(2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError, match="CUDA"):
+        forward(x, torch.zeros(2, 64), w, w, w, k=1)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not found"):
+        _lib.load.__wrapped__(str(tmp_path / "nope.so")) if hasattr(_lib.load, "__wrapped__") \
+            else _load_fresh(str(tmp_path / "nope.so"))
+
+
+def _load_fresh(path):
+    saved = _lib._lib
+    _lib._lib = None
+    try:
+        return _lib.load(path)
+    finally:
+        _lib._lib = saved
