@@ -69,6 +69,23 @@ def config_of(w, l2_note):
             "dtype_router": "f32", "l2": l2_note, "parallelism": "replicas"}
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time (all ranks call this at the same point)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
@@ -113,7 +130,7 @@ class ClockSampler:
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v})
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
         load = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
         return {"sm_mhz": statistics.median(load) if load else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
@@ -249,11 +266,7 @@ def run_ours(args, rank, world, local_rank):
                   for j in range(MOE_NUM_KERNELS)]
     for kv in kev:
         kv.close()
-    ms_max = ms
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, dev)
 
     # algorithmic work of one step, from this step's own routing counts
     cnt = counts.cpu().numpy().astype("int64")
@@ -271,7 +284,7 @@ def run_ours(args, rank, world, local_rank):
     hbm_peak = peaks["hbm_gbs"]
 
     ms_step = ms_max / args.steps
-    value = world * w.T * args.steps / (ms_max / 1e3)
+    value = job_value(world, w.T, args.steps, ms_max)
     k_up = per_kernel[4]
     achieved = flops_up / (k_up / 1e3) / 1e12
     roofline_ms = max(flops_active / (tensor_peak * 1e12), (w_bytes + act_bytes) / (hbm_peak * 1e9)) * 1e3
@@ -328,12 +341,8 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        line["e2e"] = {"value": world * w.T * ke / (ems / 1e3), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        line["e2e"] = {"value": job_value(world, w.T, ke, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": w.T * w.d * esz,
                        "d2h_bytes_per_step": w.T * w.d * esz + 4 + 4 * w.E,
                        "steps": ke, "api": "moe_forward_host_io"}

@@ -90,6 +90,12 @@ typedef struct {
   void* const* events;       /* optional cudaEvent_t[2*MOE_NUM_KERNELS]; when non-NULL,
                                 events[2i] / events[2i+1] are recorded on `stream`
                                 right before / after kernel i (NULL entries skipped) */
+  uint64_t wait_timeout_ns;  /* limit of each device-side mbarrier wait in the GEMM
+                                kernels; 0 = default (4 s). A tiny value makes the waits
+                                expire on purpose: the kernels then record
+                                MOE_ERR_DEVICE_TIMEOUT, let their in-flight copies and
+                                MMAs land, free TMEM and return (outputs undefined), and
+                                the context stays usable. */
 } moe_dims;
 
 /* Bytes of device workspace moe_forward needs for this layer (0 on invalid

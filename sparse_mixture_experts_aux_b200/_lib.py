@@ -39,6 +39,7 @@ class moe_dims(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
         ("events", ctypes.c_void_p),
+        ("wait_timeout_ns", ctypes.c_uint64),
     ]
 
 
@@ -115,7 +116,7 @@ def _ptr(t) -> int:
 
 def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, router_bias=None,
               workspace=None, workspace_bytes: int = 0, stream: int = 0, events=None,
-              gate_mode: int = 0) -> moe_dims:
+              gate_mode: int = 0, wait_timeout_ns: int = 0) -> moe_dims:
     """Fill a moe_dims. `events` is a ctypes array of cudaEvent_t handles or None."""
     dims = moe_dims()
     dims.T, dims.d, dims.d_e, dims.d_s = int(T), int(d), int(d_e), int(d_s)
@@ -125,6 +126,7 @@ def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, rou
     dims.workspace_bytes = int(workspace_bytes)
     dims.stream = int(stream) or None
     dims.events = ctypes.cast(events, ctypes.c_void_p) if events is not None else None
+    dims.wait_timeout_ns = int(wait_timeout_ns)
     return dims
 
 

@@ -18,7 +18,8 @@ namespace {
 using moe::ROW_TILE;
 
 constexpr size_t ALIGN = 1024;
-constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s per mbarrier wait
+constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;   // 4 s per mbarrier wait
+constexpr unsigned long long kDrainTimeoutNs = 2000000000ull;  // teardown waits
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -30,6 +31,7 @@ struct Plan {
   size_t esz;
   int64_t C;  // -1: no limit
   int nblk;   // routing chunks
+  int router_split;  // K chunks of the router product
   int64_t rows_max;
   size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
       o_tile_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys, total;
@@ -79,7 +81,8 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
     return o;
   };
   const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
-  p.o_logits = take(T * E * 4);
+  p.router_split = moe::simt_split_k(p.T, E, p.d);
+  p.o_logits = take(static_cast<size_t>(p.router_split) * T * E * 4);
   p.o_idx = take(TK * 4);
   p.o_gate = take(TK * 4);
   p.o_lrank = take(TK * 4);
@@ -207,10 +210,12 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   rg.N = P.E;
   rg.K = P.d;
   rg.active = 1;
+  rg.split_k = P.router_split;
   moe::SimtGroup none{};
   tm.at(0);
   {
-    dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM, 1);
+    dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM,
+              P.router_split);
     moe::simt_gemm_kernel<TX, float, float, moe::EPI_STORE_F32><<<grid, 256, 0, st>>>(rg, none);
   }
   tm.at(1);
@@ -222,7 +227,8 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
     const size_t smem = static_cast<size_t>(2) * moe::ROUTE_WARPS * P.E * 4;
     const int nv = (P.E + 31) / 32;
 #define MOE_ROUTE(NV)                                                                           \
-  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(logits, dims->router_bias, T, P.E, P.k, idx, \
+  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(logits, P.router_split, dims->router_bias, \
+                                                   T, P.E, P.k, idx, \
                                                    gate, lrank, hist, psum_part)
     if (nv <= 1) MOE_ROUTE(1);
     else if (nv <= 2) MOE_ROUTE(2);
@@ -283,6 +289,9 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
 
   uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
   const Timer tm{dims->events, st};
+  const unsigned long long wait_tmo =
+      dims->wait_timeout_ns != 0 ? static_cast<unsigned long long>(dims->wait_timeout_ns)
+                                 : kWaitTimeoutNs;
   const int T = static_cast<int>(P.T);
   int32_t* slot = reinterpret_cast<int32_t*>(ws + P.o_slot);
   int32_t* tile_start = reinterpret_cast<int32_t*>(ws + P.o_tile_start);
@@ -316,7 +325,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       if (!ok) return MOE_ERR_CUDA;
       moe::tc::TcParams tp{};
       tp.num_groups = ng;
-      tp.timeout_ns = kWaitTimeoutNs;
+      tp.timeout_ns = wait_tmo;
+      tp.drain_timeout_ns = kDrainTimeoutNs;
       tp.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
                  P.d / moe::tc::BK, P.de, h, nullptr};
       if (P.ds)
@@ -342,7 +352,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       maps.b1[1] = maps.b0[1];
       moe::tc::TcParams tp{};
       tp.num_groups = ng;
-      tp.timeout_ns = kWaitTimeoutNs;
+      tp.timeout_ns = wait_tmo;
+      tp.drain_timeout_ns = kDrainTimeoutNs;
       tp.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
                  P.d, yrows, rowgate};
       if (P.ds)
@@ -377,8 +388,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   {
     moe::SimtGroup a{}, b{};
     a = {xp, W_g, W_u, static_cast<int64_t>(P.de) * P.d, h, nullptr, tile_start, E, 0, P.de, P.d,
-         1};
-    if (P.ds) b = {xf, sg, sg + sh_n, 0, hs, nullptr, nullptr, 1, P.T, P.ds, P.d, 1};
+         1, 1};
+    if (P.ds) b = {xf, sg, sg + sh_n, 0, hs, nullptr, nullptr, 1, P.T, P.ds, P.d, 1, 1};
     const int nmax = P.de > P.ds ? P.de : P.ds;
     dim3 grid((nmax + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
@@ -390,8 +401,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   {
     moe::SimtGroup a{}, b{};
     a = {h, W_d, nullptr, static_cast<int64_t>(P.d) * P.de, yrows, rowgate, tile_start, E, 0, P.d,
-         P.de, 1};
-    if (P.ds) b = {hs, sg + 2 * sh_n, nullptr, 0, ys, nullptr, nullptr, 1, P.T, P.d, P.ds, 1};
+         P.de, 1, 1};
+    if (P.ds) b = {hs, sg + 2 * sh_n, nullptr, 0, ys, nullptr, nullptr, 1, P.T, P.d, P.ds, 1, 1};
     dim3 grid((P.d + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
     tm.at(10);

@@ -27,16 +27,28 @@ struct SimtGroup {
   const void* B0;           // expert e at B0 + e * b_stride  ([N, K] each)
   const void* B1;           // second operand of the SwiGLU (up projection)
   int64_t b_stride;         // elements between experts
-  void* C;                  // [rows, N]
+  void* C;                  // [rows, N]; with split_k > 1: [split_k][rows][N] partial sums
   const float* row_scale;   // EPI_SCALE: multiplier per row (NULL = 1)
   const int32_t* tile_start;// grouped rows: [E + 1] segment starts in ROW_TILE units; NULL = dense
   int E;
   int64_t rows;             // dense: number of valid rows
   int N, K;
   int active;               // 0: this grid z-slice does nothing
+  int split_k;              // > 1 (EPI_STORE_F32 only): grid z splits K into equal chunks
 };
 
-constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 32;
+
+// Number of K chunks for a dense fp32-output product of rows x N x K: enough
+// blocks to fill the GPU several times over, chunks of at least 256 and a
+// multiple of SG_BK. Depends only on the shape, so the workspace size does too.
+inline int simt_split_k(int64_t rows, int N, int K) {
+  const int64_t blocks = ((N + SG_BN - 1) / SG_BN) * ((rows + SG_BM - 1) / SG_BM);
+  int split = 1;
+  while (blocks * split < 600 && (K % (2 * split * SG_BK)) == 0 && K / (2 * split) >= 256)
+    split *= 2;
+  return split;
+}
 
 template <typename TA>
 __device__ __forceinline__ void load4(const TA* p, float* f);
@@ -53,10 +65,19 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
   f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
 }
 
+// 64x64 output tile per 256-thread block, 4x4 outputs per thread, K tiles of
+// 32 staged in shared memory; the next tile's global loads are issued before
+// the current tile is consumed. Each K tile is summed into a fresh partial
+// that is then added to the running total (blocked summation), which keeps
+// the rounding error of a long dot product well below one sequential chain.
 template <typename TA, typename TB, typename TC, int EPI>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup g1) {
-  const SimtGroup g = blockIdx.z == 0 ? g0 : g1;
+  const bool splitting = g0.split_k > 1;
+  const SimtGroup g = (splitting || blockIdx.z == 0) ? g0 : g1;
   if (!g.active) return;
+  const int split = splitting ? (int)blockIdx.z : 0;
+  const int k_len = splitting ? g.K / g.split_k : g.K;
+  const int k_begin = split * k_len;
   const int n0 = blockIdx.x * SG_BN;
   const int64_t m0 = (int64_t)blockIdx.y * SG_BM;
   if (n0 >= g.N) return;
@@ -77,11 +98,11 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
     m_end = g.rows;
   }
   constexpr int NB = (EPI == EPI_SWIGLU) ? 2 : 1;
-  __shared__ float As[SG_BK][SG_BM + 4];
-  __shared__ float Bs[NB][SG_BK][SG_BN + 4];
+  __shared__ __align__(16) float As[SG_BK][SG_BM + 4];
+  __shared__ __align__(16) float Bs[NB][SG_BK][SG_BN + 4];
 
   const int tid = threadIdx.x;
-  const int lr = tid >> 2, lk = (tid & 3) * 4;
+  const int lr = tid >> 2, lk = (tid & 3) * 8;  // row within the tile, first of 8 K elements
   const int ty = tid >> 4, tx = tid & 15;
   const TA* A = reinterpret_cast<const TA*>(g.A);
   const TB* Bp[2] = {reinterpret_cast<const TB*>(g.B0) + (int64_t)e * g.b_stride,
@@ -96,23 +117,35 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
 
   const int64_t arow = m0 + lr;
   const int brow = n0 + lr;
-  for (int k0 = 0; k0 < g.K; k0 += SG_BK) {
-    float f[4] = {0.f, 0.f, 0.f, 0.f};
-    if (arow < m_end) load4<TA>(A + arow * g.K + k0 + lk, f);
+  const bool a_ok = arow < m_end, b_ok = brow < g.N;
+  float fa[8], fb[NB][8];
+  auto fetch = [&](int k0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) As[lk + i][lr] = f[i];
+    for (int i = 0; i < 8; ++i) fa[i] = 0.f;
+    if (a_ok) {
+      load4<TA>(A + arow * g.K + k0 + lk, fa);
+      load4<TA>(A + arow * g.K + k0 + lk + 4, fa + 4);
+    }
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      float h[4] = {0.f, 0.f, 0.f, 0.f};
-      if (brow < g.N) load4<TB>(Bp[b] + (int64_t)brow * g.K + k0 + lk, h);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) Bs[b][lk + i][lr] = h[i];
+      for (int i = 0; i < 8; ++i) fb[b][i] = 0.f;
+      if (b_ok) {
+        load4<TB>(Bp[b] + (int64_t)brow * g.K + k0 + lk, fb[b]);
+        load4<TB>(Bp[b] + (int64_t)brow * g.K + k0 + lk + 4, fb[b] + 4);
+      }
     }
+  };
+  fetch(k_begin);
+  for (int k0 = k_begin; k0 < k_begin + k_len; k0 += SG_BK) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) As[lk + i][lr] = fa[i];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Bs[b][lk + i][lr] = fb[b][i];
     __syncthreads();
-    // Blocked summation: each K tile is summed into a fresh partial that is
-    // then added to the running total, which keeps the rounding error of a
-    // long dot product (d up to thousands) about sqrt(SG_BK) times smaller
-    // than one sequential chain.
+    if (k0 + SG_BK < k_begin + k_len) fetch(k0 + SG_BK);  // in flight during the compute below
     float part[NB][4][4];
 #pragma unroll
     for (int b = 0; b < NB; ++b)
@@ -143,7 +176,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
     __syncthreads();
   }
 
-  TC* C = reinterpret_cast<TC*>(g.C);
+  TC* C = reinterpret_cast<TC*>(g.C) + (splitting ? (int64_t)split * g.rows * g.N : 0);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t m = m0 + ty * 4 + i;
@@ -192,7 +225,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 template <int NV>
 __global__ void __launch_bounds__(256) route_kernel(
-    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    float* __restrict__ logits, int splits, const float* __restrict__ bias, int T, int E, int k,
     int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int32_t* __restrict__ lrank_out,
     int32_t* __restrict__ hist, double* __restrict__ psum_part) {
   extern __shared__ uint32_t route_smem[];
@@ -216,7 +249,8 @@ __global__ void __launch_bounds__(256) route_kernel(
   for (int j = 0; j < 32; ++j) {
     const int t = t_warp0 + j;
     if (t >= T) break;  // warp-uniform
-    const float* row = logits + (size_t)t * E;
+    float* row = logits + (size_t)t * E;
+    const size_t split_stride = (size_t)T * E;
     float v[NV];
     uint32_t removed = 0u;
     float m = -INFINITY;
@@ -224,7 +258,10 @@ __global__ void __launch_bounds__(256) route_kernel(
     for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
       if (e < E) {
-        v[i] = row[e] + bv[i];
+        float r = row[e];
+        for (int sp = 1; sp < splits; ++sp) r += row[sp * split_stride + e];  // fixed order
+        if (splits > 1) row[e] = r;  // the summed logit, for readers of the workspace
+        v[i] = r + bv[i];
         m = fmaxf(m, v[i]);
       } else {
         v[i] = -INFINITY;

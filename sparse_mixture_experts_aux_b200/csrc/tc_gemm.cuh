@@ -61,7 +61,8 @@ struct TcGroup {
 struct TcParams {
   TcGroup g[2];
   int num_groups;
-  unsigned long long timeout_ns;
+  unsigned long long timeout_ns;        // limit of each pipeline wait
+  unsigned long long drain_timeout_ns;  // limit of the teardown waits for work in flight
 };
 
 struct TcMaps {
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       p.num_groups > 1 ? (long long)p.g[1].n_tiles * ((p.g[1].rows + BM - 1) / BM) : 0;
   const long long total = tiles0 + tiles1;
   const unsigned long long tmo = p.timeout_ns;
+  const unsigned long long drain_tmo = p.drain_timeout_ns;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
-          if ((issued >> s) & 1u) wait_drain(full_bar(s), (last_par >> s) & 1u, tmo);
+          if ((issued >> s) & 1u) wait_drain(full_bar(s), (last_par >> s) & 1u, drain_tmo);
       }
     }
   } else if (warp == 1) {
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (acc == 0u) acc_phase ^= 1u;
       }
       tc_commit(done_bar);  // every MMA issued above has completed once this fires
-      wait_drain(done_bar, 0u, tmo);
+      wait_drain(done_bar, 0u, drain_tmo);
     }
   } else {
     // ------------------------------------------------------------ epilogue
