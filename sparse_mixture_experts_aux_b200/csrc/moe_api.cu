@@ -12,6 +12,7 @@
 #include "router.cuh"
 #include "permute.cuh"
 #include "tc_gemm.cuh"
+#include "tc2_gemm.cuh"
 
 namespace {
 
@@ -31,10 +32,11 @@ struct Plan {
   size_t esz;
   int64_t C;  // -1: no limit
   int nblk;   // routing chunks
-  int router_split;  // K chunks of the router product
+  int router_split;    // K chunks of the router product
+  bool router_narrow;  // few experts, many tokens: warp-per-token-group router kernel
   int64_t rows_max;
   size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
-      o_tile_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys, total;
+      o_tile_start, o_pair_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys, total;
 };
 
 int64_t capacity_of(int64_t T, int E, int k, float cf) {
@@ -81,7 +83,8 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
     return o;
   };
   const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
-  p.router_split = moe::simt_split_k(p.T, E, p.d);
+  p.router_narrow = E <= 16 && p.T >= 1024;
+  p.router_split = p.router_narrow ? 1 : moe::simt_split_k(p.T, E, p.d);
   p.o_logits = take(static_cast<size_t>(p.router_split) * T * E * 4);
   p.o_idx = take(TK * 4);
   p.o_gate = take(TK * 4);
@@ -92,6 +95,7 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   p.o_psum_part = take(static_cast<size_t>(p.nblk) * moe::ROUTE_WARPS * E * 8);
   p.o_probsum = take(static_cast<size_t>(E) * 8);
   p.o_tile_start = take(static_cast<size_t>(E + 1) * 4);
+  p.o_pair_start = take(static_cast<size_t>(E + 1) * 4);
   p.o_rowgate = take(R * 4);
   p.o_xp = take(R * p.d * p.esz);
   p.o_h = take(R * p.de * p.esz);
@@ -108,6 +112,7 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  int pair_clusters[2] = {0, 0};  // co-resident 2-CTA clusters of each pair GEMM kernel
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -119,7 +124,37 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-moe_status device_setup(int* num_sms) {
+template <int EPI>
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(moe::tc2::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = moe::tc2::SMEM_BYTES;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <int EPI>
+bool pair_setup(int num_sms, int* clusters) {
+  auto kern = moe::tc2::tc2_grouped_gemm_kernel<EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           moe::tc2::SMEM_BYTES) != cudaSuccess)
+    return false;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config<EPI>(num_sms / 2, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return false;
+  *clusters = n < num_sms / 2 ? n : num_sms / 2;
+  return true;
+}
+
+moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_dev_mutex);
@@ -142,6 +177,9 @@ moe_status device_setup(int* num_sms) {
         cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
+        !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
+      return MOE_ERR_CUDA;
     const int rs = 2 * moe::ROUTE_WARPS * moe::tc::MAX_E * 4;
     if (cudaFuncSetAttribute(moe::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              rs) != cudaSuccess ||
@@ -151,6 +189,10 @@ moe_status device_setup(int* num_sms) {
     di.ready = true;
   }
   *num_sms = di.num_sms;
+  if (pair_clusters != nullptr) {
+    pair_clusters[0] = di.pair_clusters[0];
+    pair_clusters[1] = di.pair_clusters[1];
+  }
   return MOE_OK;
 }
 
@@ -193,6 +235,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   double* psum_part = reinterpret_cast<double*>(ws + P.o_psum_part);
   double* probsum = reinterpret_cast<double*>(ws + P.o_probsum);
   int32_t* tile_start = reinterpret_cast<int32_t*>(ws + P.o_tile_start);
+  int32_t* pair_start = reinterpret_cast<int32_t*>(ws + P.o_pair_start);
   float* rowgate = reinterpret_cast<float*>(ws + P.o_rowgate);
   TX* xp = reinterpret_cast<TX*>(ws + P.o_xp);
   const int T = static_cast<int>(P.T);
@@ -213,7 +256,14 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   rg.split_k = P.router_split;
   moe::SimtGroup none{};
   tm.at(0);
-  {
+  if (P.router_narrow) {
+    const int warps = (T + moe::ROUTER_TOK - 1) / moe::ROUTER_TOK;
+    const int blocks = (warps + 7) / 8;
+    if (P.E <= 8)
+      moe::router_narrow_kernel<TX, 1><<<blocks, 256, 0, st>>>(x, W_r, T, P.d, P.E, logits);
+    else
+      moe::router_narrow_kernel<TX, 2><<<blocks, 256, 0, st>>>(x, W_r, T, P.d, P.E, logits);
+  } else {
     dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM,
               P.router_split);
     moe::simt_gemm_kernel<TX, float, float, moe::EPI_STORE_F32><<<grid, 256, 0, st>>>(rg, none);
@@ -244,7 +294,8 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   // (2) scan: counts, capacity, segment offsets, aux
   tm.at(4);
   moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk * moe::ROUTE_WARPS, P.E,
-                                       P.T, P.k, P.C, counts, base, tile_start, probsum, aux);
+                                       P.T, P.k, P.C, counts, base, tile_start, pair_start,
+                                       probsum, aux);
   tm.at(5);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
 
@@ -283,8 +334,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   if (dims->workspace == nullptr || !aligned(dims->workspace, 256) ||
       dims->workspace_bytes < P.total)
     return MOE_ERR_WORKSPACE;
-  int num_sms = 0;
-  s = device_setup(&num_sms);
+  int num_sms = 0, pair_clusters[2] = {0, 0};
+  s = device_setup(&num_sms, pair_clusters);
   if (s != MOE_OK) return s;
 
   uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
@@ -311,57 +362,107 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     const size_t sh_n = static_cast<size_t>(P.ds) * P.d;
     const int ng = P.ds ? 2 : 1;
 
-    // (4) gate/up projection + SwiGLU
+    // (4) gate/up projection + SwiGLU, (5) down projection scaled by the gates.
+    // CTA-pair tiles (256 rows) cut the operand traffic per SM by a third but
+    // pair up the 128-row tiles of each expert, so an expert with an odd tile
+    // count computes one idle half-tile. They are used where experts get many
+    // rows: down (long K, few N tiles) from 512 rows per expert, gate/up from 2048.
+    const int64_t rows_per_expert = P.T * P.k / E;
+#if defined(MOE_FORCE_1CTA)
+    const bool pair_up = false, pair_down = false;
+#elif defined(MOE_FORCE_PAIR)
+    const bool pair_up = true, pair_down = true;
+#else
+    const bool pair_up = rows_per_expert >= 2048;
+    const bool pair_down = rows_per_expert >= 512;
+#endif
+    int32_t* pair_start = reinterpret_cast<int32_t*>(ws + P.o_pair_start);
+    constexpr int HB = 128;  // rows of B each CTA of a pair loads
+    constexpr int BNp = moe::tc2::BN;
+    cudaLaunchAttribute attr[1];
     {
-      moe::tc::TcMaps maps;
-      memset(&maps, 0, sizeof(maps));
-      bool ok = encode_map(&maps.a[0], xp, P.d, P.rows_max, 1, moe::tc::BM, 2) &&
-                encode_map(&maps.b0[0], W_g, P.d, P.de, E, moe::tc::BN / 2, 3) &&
-                encode_map(&maps.b1[0], W_u, P.d, P.de, E, moe::tc::BN / 2, 3);
+      const int brows = pair_up ? HB : moe::tc::BN / 2;
+      moe::tc::TcMaps up;
+      memset(&up, 0, sizeof(up));
+      bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, moe::tc::BM, 2) &&
+                encode_map(&up.b0[0], W_g, P.d, P.de, E, brows, 3) &&
+                encode_map(&up.b1[0], W_u, P.d, P.de, E, brows, 3);
       if (P.ds)
-        ok = ok && encode_map(&maps.a[1], x, P.d, P.T, 1, moe::tc::BM, 2) &&
-             encode_map(&maps.b0[1], sg, P.d, P.ds, 1, moe::tc::BN / 2, 3) &&
-             encode_map(&maps.b1[1], sg + sh_n, P.d, P.ds, 1, moe::tc::BN / 2, 3);
+        ok = ok && encode_map(&up.a[1], x, P.d, P.T, 1, moe::tc::BM, 2) &&
+             encode_map(&up.b0[1], sg, P.d, P.ds, 1, brows, 3) &&
+             encode_map(&up.b1[1], sg + sh_n, P.d, P.ds, 1, brows, 3);
       if (!ok) return MOE_ERR_CUDA;
-      moe::tc::TcParams tp{};
-      tp.num_groups = ng;
-      tp.timeout_ns = wait_tmo;
-      tp.drain_timeout_ns = kDrainTimeoutNs;
-      tp.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
-                 P.d / moe::tc::BK, P.de, h, nullptr};
-      if (P.ds)
-        tp.g[1] = {nullptr, 1, T, (P.ds + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
-                   P.d / moe::tc::BK, P.ds, hs, nullptr};
       tm.at(8);
-      moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>
-          <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(maps, tp);
+      if (pair_up) {
+        moe::tc2::Tc2Params tu{};
+        tu.num_groups = ng;
+        tu.timeout_ns = wait_tmo;
+        tu.drain_timeout_ns = kDrainTimeoutNs;
+        tu.g[0] = {tile_start, pair_start, E, 0, (P.de + BNp / 2 - 1) / (BNp / 2),
+                   P.d / moe::tc::BK, P.de, h, nullptr};
+        if (P.ds)
+          tu.g[1] = {nullptr, nullptr, 1, T, (P.ds + BNp / 2 - 1) / (BNp / 2), P.d / moe::tc::BK,
+                     P.ds, hs, nullptr};
+        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SWIGLU_TC>(pair_clusters[0], st, attr);
+        if (cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>,
+                               up, tu) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      } else {
+        moe::tc::TcParams tp{};
+        tp.num_groups = ng;
+        tp.timeout_ns = wait_tmo;
+        tp.drain_timeout_ns = kDrainTimeoutNs;
+        tp.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                   P.d / moe::tc::BK, P.de, h, nullptr};
+        if (P.ds)
+          tp.g[1] = {nullptr, 1, T, (P.ds + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                     P.d / moe::tc::BK, P.ds, hs, nullptr};
+        moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>
+            <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(up, tp);
+      }
       tm.at(9);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     }
-    // (5) down projection, scaled by the assignment's gate
     {
-      moe::tc::TcMaps maps;
-      memset(&maps, 0, sizeof(maps));
-      bool ok = encode_map(&maps.a[0], h, P.de, P.rows_max, 1, moe::tc::BM, 2) &&
-                encode_map(&maps.b0[0], W_d, P.de, P.d, E, moe::tc::BN, 3);
+      const int brows = pair_down ? HB : moe::tc::BN;
+      moe::tc::TcMaps dn;
+      memset(&dn, 0, sizeof(dn));
+      bool ok = encode_map(&dn.a[0], h, P.de, P.rows_max, 1, moe::tc::BM, 2) &&
+                encode_map(&dn.b0[0], W_d, P.de, P.d, E, brows, 3);
       if (P.ds)
-        ok = ok && encode_map(&maps.a[1], hs, P.ds, P.T, 1, moe::tc::BM, 2) &&
-             encode_map(&maps.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, moe::tc::BN, 3);
+        ok = ok && encode_map(&dn.a[1], hs, P.ds, P.T, 1, moe::tc::BM, 2) &&
+             encode_map(&dn.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, brows, 3);
       if (!ok) return MOE_ERR_CUDA;
-      maps.b1[0] = maps.b0[0];
-      maps.b1[1] = maps.b0[1];
-      moe::tc::TcParams tp{};
-      tp.num_groups = ng;
-      tp.timeout_ns = wait_tmo;
-      tp.drain_timeout_ns = kDrainTimeoutNs;
-      tp.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
-                 P.d, yrows, rowgate};
-      if (P.ds)
-        tp.g[1] = {nullptr, 1, T, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.ds / moe::tc::BK, P.d,
-                   ys, nullptr};
+      dn.b1[0] = dn.b0[0];
+      dn.b1[1] = dn.b0[1];
       tm.at(10);
-      moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>
-          <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(maps, tp);
+      if (pair_down) {
+        moe::tc2::Tc2Params td{};
+        td.num_groups = ng;
+        td.timeout_ns = wait_tmo;
+        td.drain_timeout_ns = kDrainTimeoutNs;
+        td.g[0] = {tile_start, pair_start, E, 0, (P.d + BNp - 1) / BNp, P.de / moe::tc::BK, P.d,
+                   yrows, rowgate};
+        if (P.ds)
+          td.g[1] = {nullptr, nullptr, 1, T, (P.d + BNp - 1) / BNp, P.ds / moe::tc::BK, P.d, ys,
+                     nullptr};
+        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SCALE_TC>(pair_clusters[1], st, attr);
+        if (cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
+                               dn, td) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      } else {
+        moe::tc::TcParams tp{};
+        tp.num_groups = ng;
+        tp.timeout_ns = wait_tmo;
+        tp.drain_timeout_ns = kDrainTimeoutNs;
+        tp.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
+                   P.d, yrows, rowgate};
+        if (P.ds)
+          tp.g[1] = {nullptr, 1, T, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.ds / moe::tc::BK,
+                     P.d, ys, nullptr};
+        moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>
+            <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(dn, tp);
+      }
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     }

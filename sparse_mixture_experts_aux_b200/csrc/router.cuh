@@ -202,6 +202,86 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
 }
 
 // ---------------------------------------------------------------------------
+// Router logits for few experts (E <= 8 * NG): r[t, e] = sum_j x[t, j] W_r[e, j].
+// Memory-bound on x, so there is no output tile to waste: each warp owns
+// ROUTER_TOK consecutive tokens over the whole of K; lane l takes the 8
+// consecutive elements at 8l + 256i of every row, multiplies them by the same
+// slice of every router row (read through L1, shared by all warps), and keeps
+// one fp32 partial per (token, expert). The 32 lane partials of each output
+// are then summed by a fixed butterfly, so the result is deterministic. Each
+// lane's chain has d/32 terms.
+// ---------------------------------------------------------------------------
+constexpr int ROUTER_TOK = 4;
+
+template <typename TA>
+__device__ __forceinline__ void load8(const TA* p, float* f);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  Vec16<__nv_bfloat16>::unpack(ld_nc_v4(p), f);
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* f) {
+  Vec16<float>::unpack(ld_nc_v4(p), f);
+  Vec16<float>::unpack(ld_nc_v4(p + 4), f + 4);
+}
+
+template <typename TA, int NG>  // NG groups of 8 experts
+__global__ void __launch_bounds__(256) router_narrow_kernel(const TA* __restrict__ x,
+                                                            const float* __restrict__ W_r, int T,
+                                                            int d, int E,
+                                                            float* __restrict__ logits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = (blockIdx.x * (blockDim.x >> 5) + warp) * ROUTER_TOK;
+  if (t0 >= T) return;  // warp-uniform
+  float acc[ROUTER_TOK][NG * 8];
+#pragma unroll
+  for (int t = 0; t < ROUTER_TOK; ++t)
+#pragma unroll
+    for (int e = 0; e < NG * 8; ++e) acc[t][e] = 0.f;
+  for (int j = lane * 8; j < d; j += 256) {
+    float xv[ROUTER_TOK][8];
+#pragma unroll
+    for (int t = 0; t < ROUTER_TOK; ++t) {
+      if (t0 + t < T) load8<TA>(x + (size_t)(t0 + t) * d + j, xv[t]);
+      else
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xv[t][i] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < NG * 8; ++e) {
+      if (e < E) {
+        float wv[8];
+        load8<float>(W_r + (size_t)e * d + j, wv);
+#pragma unroll
+        for (int t = 0; t < ROUTER_TOK; ++t) {
+          float part = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part = fmaf(xv[t][i], wv[i], part);
+          acc[t][e] += part;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < ROUTER_TOK; ++t)
+#pragma unroll
+    for (int e = 0; e < NG * 8; ++e) {
+      float v = acc[t][e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      acc[t][e] = v;
+    }
+  if (lane == 0) {
+#pragma unroll
+    for (int t = 0; t < ROUTER_TOK; ++t)
+      if (t0 + t < T)
+#pragma unroll
+        for (int e = 0; e < NG * 8; ++e)
+          if (e < E) logits[(size_t)(t0 + t) * E + e] = acc[t][e];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Routing: one warp per token, ROUTE_CHUNK tokens per block.
 //   softmax over all E logits (+ optional bias), per-expert probability sums
 //   accumulated in fp64 in a fixed order; top-k by k rounds of a warp argmax
@@ -246,11 +326,32 @@ __global__ void __launch_bounds__(256) route_kernel(
     bv[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   }
 
+  // The next token's logits are loaded (and their K-split partials summed, in
+  // a fixed order) while the current token is processed.
+  const size_t split_stride = (size_t)T * E;
+  float nxt[NV];
+  auto load_logits = [&](int t) {
+    const float* row = logits + (size_t)t * E;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      float r = 0.f;
+      if (e < E) {
+        r = row[e];
+        for (int sp = 1; sp < splits; ++sp) r += row[sp * split_stride + e];
+      }
+      nxt[i] = r;
+    }
+  };
+  if (t_warp0 < T) load_logits(t_warp0);
   for (int j = 0; j < 32; ++j) {
     const int t = t_warp0 + j;
     if (t >= T) break;  // warp-uniform
+    float raw[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) raw[i] = nxt[i];
+    if (j + 1 < 32 && t + 1 < T) load_logits(t + 1);
     float* row = logits + (size_t)t * E;
-    const size_t split_stride = (size_t)T * E;
     float v[NV];
     uint32_t removed = 0u;
     float m = -INFINITY;
@@ -258,10 +359,8 @@ __global__ void __launch_bounds__(256) route_kernel(
     for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
       if (e < E) {
-        float r = row[e];
-        for (int sp = 1; sp < splits; ++sp) r += row[sp * split_stride + e];  // fixed order
-        if (splits > 1) row[e] = r;  // the summed logit, for readers of the workspace
-        v[i] = r + bv[i];
+        if (splits > 1) row[e] = raw[i];  // the summed logit, for readers of the workspace
+        v[i] = raw[i] + bv[i];
         m = fmaxf(m, v[i]);
       } else {
         v[i] = -INFINITY;
@@ -350,13 +449,15 @@ __global__ void __launch_bounds__(256) route_kernel(
 //   counts[e]    = routed assignments to e (before the capacity cut)
 //   kept_e       = min(counts[e], C); segment of ceil(kept_e / ROW_TILE) tiles
 //   tile_start   = exclusive scan of the segment sizes; tile_start[E] = total
+//   pair_start   = exclusive scan of ceil(segment tiles / 2) (CTA-pair tiles)
 //   probsum[e]   = sum of the probability partials, fp64, fixed order
 //   aux          = E * sum_e (counts_e / (T k)) (probsum_e / T), fp64, fixed tree
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) scan_kernel(
     const int32_t* __restrict__ hist, int nblk, const double* __restrict__ psum_part, int nparts,
     int E, int64_t T, int k, int64_t C, int32_t* __restrict__ counts, int32_t* __restrict__ base,
-    int32_t* __restrict__ tile_start, double* __restrict__ probsum, float* __restrict__ aux) {
+    int32_t* __restrict__ tile_start, int32_t* __restrict__ pair_start,
+    double* __restrict__ probsum, float* __restrict__ aux) {
   __shared__ int s_scan[2][1024];
   __shared__ double s_sum[1024];
   const int e = threadIdx.x;
@@ -388,6 +489,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(
   }
   if (e < E) tile_start[e] = s_scan[cur][e] - tiles;
   if (e == E - 1) tile_start[E] = s_scan[cur][e];
+  // the same scan over pairs of tiles (a CTA pair computes two tiles of one expert)
+  const int pairs = (tiles + 1) / 2;
+  __syncthreads();
+  s_scan[0][e] = pairs;
+  cur = 0;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int v = s_scan[cur][e] + (e >= off ? s_scan[cur][e - off] : 0);
+    s_scan[cur ^ 1][e] = v;
+    cur ^= 1;
+    __syncthreads();
+  }
+  if (e < E) pair_start[e] = s_scan[cur][e] - pairs;
+  if (e == E - 1) pair_start[E] = s_scan[cur][e];
   for (int half = 512; half > 0; half >>= 1) {  // fixed-shape tree sum
     if (e < half) s_sum[e] += s_sum[e + half];
     __syncthreads();

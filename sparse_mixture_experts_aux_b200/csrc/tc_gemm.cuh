@@ -108,7 +108,8 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 0u) {
+    // try_wait itself suspends for a while, so check on the first re-poll too
+    if ((it & 127u) == 1u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         atomicOr(&g_dev_error, DEVERR_TIMEOUT);
@@ -127,7 +128,7 @@ __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity,
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 0u && globaltimer_ns() - t0 > timeout_ns) {
+    if ((it & 127u) == 1u && globaltimer_ns() - t0 > timeout_ns) {
       atomicOr(&g_dev_error, DEVERR_TIMEOUT);
       return false;
     }

@@ -36,7 +36,13 @@ def run_oracle(w: Workload, inp: dict, rows=None) -> O.OracleResult:
     shared = None
     if w.d_s:
         shared = tuple(t.cpu() for t in split_shared(inp["W_shared"], w.d, w.d_s))
-    return O.moe_forward(x, inp["W_r"].cpu(), expert, w.k, w.capacity_factor, bias, shared, rows)
+    return O.moe_forward(x, inp["W_r"].cpu(), expert, w.k, layer_capacity_factor(w), bias, shared,
+                         rows)
+
+
+def layer_capacity_factor(w: Workload) -> float:
+    """The capacity factor as the layer receives it: the C ABI takes an fp32."""
+    return float(np.float32(w.capacity_factor))
 
 
 def expected_slot_pos(ref: O.OracleResult, E: int) -> tuple:

@@ -56,8 +56,12 @@ def test_capacity_matches_page_example(lib):
 
 def test_capacity_agrees_with_oracle_formula(lib):
     from oracle import moe_oracle as O
-    for T, E, k, cf in [(1000, 7, 3, 1.1), (333, 5, 2, 0.37), (4096, 64, 1, 2.0), (17, 3, 1, 0.99)]:
-        assert _lib.moe_capacity(T, E, k, cf) == O.capacity_limit(cf, T, k, E)
+    import numpy as np
+    # the layer takes the factor as an fp32; the oracle is given that same value
+    for T, E, k, cf in [(1000, 7, 3, 1.1), (333, 5, 2, 0.37), (4096, 64, 1, 2.0), (17, 3, 1, 0.99),
+                        (2600, 4, 1, 0.9)]:
+        cf32 = float(np.float32(cf))
+        assert _lib.moe_capacity(T, E, k, cf) == O.capacity_limit(cf32, T, k, E)
 
 
 def _dims(**kw):

@@ -29,6 +29,14 @@ SMALL = [
     Workload("bf16 shared+capacity", 700, 256, 8, 256, 2, d_s=256, capacity_factor=0.8, seed=21),
     Workload("fp32 shared+capacity", 333, 128, 8, 96, 2, "f32", d_s=64, capacity_factor=0.7, seed=22),
     Workload("fp32 ragged", 257, 96, 5, 160, 3, "f32", seed=23),
+    # >= 512 routed rows per expert run the down GEMM on CTA pairs (cta_group::2),
+    # >= 2048 the gate/up GEMM as well
+    Workload("pair odd tile counts", 4300, 256, 2, 320, 1, seed=24),
+    Workload("pair shared expert", 4200, 256, 2, 256, 1, d_s=128, seed=25),
+    Workload("pair both GEMMs k=2", 2200, 256, 2, 192, 2, seed=28),
+    Workload("pair down only", 1100, 256, 2, 320, 1, seed=29),
+    Workload("pair down N tail d=320", 1300, 320, 2, 256, 2, seed=26),
+    Workload("pair capacity", 2600, 256, 4, 192, 1, capacity_factor=0.9, zipf_bias=True, seed=27),
 ]
 
 
