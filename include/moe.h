@@ -60,7 +60,9 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2,    /* valid layer this build does not run (see limits below) */
   MOE_ERR_WORKSPACE = 3,      /* workspace null, too small or misaligned */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
-  MOE_ERR_DEVICE_TIMEOUT = 5  /* a device-side bounded wait gave up (moe_get_device_status) */
+  MOE_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up (moe_get_device_status) */
+  MOE_ERR_SCRATCH_LIMIT = 6   /* moe_forward_no_alloc: the layer needs more scratch than
+                                 MOE_NO_ALLOC_WORKSPACE_BYTES */
 } moe_status;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
@@ -172,6 +174,48 @@ MOE_API moe_status moe_get_device_status(void);
 
 /* Static, human-readable name of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
+
+/*
+ * moe_forward for callers that cannot allocate device memory. The pages have
+ * no counterpart: this is a deployment entry point, not part of the method.
+ *
+ * Who needs it: code that runs inside a host which owns the device memory,
+ * e.g. a plugin loaded into an inference server that has reserved all free
+ * device memory for its own pool (a cudaMalloc there fails or would steal from
+ * the pool), or a plain C caller with no allocator of its own. Such callers
+ * cannot provide moe_forward's caller-owned workspace.
+ *
+ * Instead this call uses one scratch array of MOE_NO_ALLOC_WORKSPACE_BYTES
+ * (64 MiB) that lives in the library itself as a statically sized device
+ * array: every GPU that loads the library holds it until the process exits.
+ * That covers, for example, the Mixtral-shaped layer (d=4096, E=8,
+ * d_e=14336, k=2) at T <= 128 tokens per call. The call allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Arguments and results are exactly those of moe_forward, except that
+ * dims->workspace and dims->workspace_bytes are ignored. Inputs and outputs
+ * are still caller-owned device memory.
+ *
+ * Errors: those of moe_forward, plus MOE_ERR_SCRATCH_LIMIT, returned before
+ * anything is enqueued, when moe_workspace_size() for this layer exceeds
+ * MOE_NO_ALLOC_WORKSPACE_BYTES.
+ *
+ * Set-up: the first call on each device looks up the device address of the
+ * scratch array (cudaGetSymbolAddress) with that device current, and caches
+ * it. Make that first call before any stream capture.
+ *
+ * Sharing: every call, on every stream, uses the same scratch array, which
+ * keeps the previous call's contents. The pass writes every scratch byte it
+ * later reads, so nothing has to start at zero. Calls that overlap on the GPU
+ * (for example, concurrent calls on two streams) race on the scratch and
+ * produce undefined results. Serialise them, e.g. on one stream.
+ */
+#define MOE_NO_ALLOC_WORKSPACE_BYTES ((size_t)64 << 20)
+MOE_API moe_status moe_forward_no_alloc(const moe_dims* dims,
+                                        const void* x, const float* W_r, const void* W_g,
+                                        const void* W_u, const void* W_d, const void* W_shared,
+                                        int E, int k, float capacity_factor,
+                                        void* y, float* aux, int32_t* counts);
 
 #ifdef __cplusplus
 }

@@ -17,13 +17,16 @@ MOE_ERR_UNSUPPORTED = 2
 MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_SCRATCH_LIMIT = 6
+MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_NUM_KERNELS = 7
 KERNEL_NAMES = ("router_logits", "route", "scan", "scatter", "gate_up_swiglu", "down_scale", "combine")
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_forward", "moe_forward_host_io",
-            "moe_workspace_layout", "moe_get_device_status", "moe_status_string")
+            "moe_workspace_layout", "moe_get_device_status", "moe_status_string",
+            "moe_forward_no_alloc")
 
 
 class moe_dims(ctypes.Structure):
@@ -88,6 +91,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_forward_host_io.argtypes = [P(moe_dims), vp, vp, vp, vp, vp, vp, vp, i32, i32, f32,
                                         vp, vp, vp, vp, vp, vp]
     lib.moe_forward_host_io.restype = i32
+    lib.moe_forward_no_alloc.argtypes = [P(moe_dims), vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp,
+                                         vp]
+    lib.moe_forward_no_alloc.restype = i32
     lib.moe_workspace_layout.argtypes = [P(moe_dims), i32, i32, f32, P(moe_workspace_layout_t)]
     lib.moe_workspace_layout.restype = i32
     lib.moe_get_device_status.argtypes = []
@@ -165,6 +171,17 @@ def moe_forward_host_io(dims: moe_dims, x_host, x_dev, W_r, W_g, W_u, W_d, W_sha
                                     _ptr(aux_host), _ptr(counts_dev), _ptr(counts_host))
     if check and st != MOE_OK:
         raise MoeError(st, "moe_forward_host_io")
+    return st
+
+
+def moe_forward_no_alloc(dims: moe_dims, x, W_r, W_g, W_u, W_d, W_shared, E: int, k: int,
+                         capacity_factor: float, y, aux, counts, check: bool = True) -> int:
+    """moe_forward on the library's static scratch; dims.workspace is ignored."""
+    st = load().moe_forward_no_alloc(_ref(dims), _ptr(x), _ptr(W_r), _ptr(W_g), _ptr(W_u),
+                                     _ptr(W_d), _ptr(W_shared), E, k, capacity_factor, _ptr(y),
+                                     _ptr(aux), _ptr(counts))
+    if check and st != MOE_OK:
+        raise MoeError(st, "moe_forward_no_alloc")
     return st
 
 

@@ -196,6 +196,29 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch of moe_forward_no_alloc: a statically sized device array, so the
+// call itself allocates nothing. In host code `g_no_alloc_scratch` only names
+// the symbol; its device address comes from cudaGetSymbolAddress, looked up
+// once per device with that device current.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_no_alloc_scratch[MOE_NO_ALLOC_WORKSPACE_BYTES];
+void* g_no_alloc_ptr[kMaxDevices] = {};
+
+moe_status no_alloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_no_alloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_no_alloc_scratch) != cudaSuccess || ptr == nullptr)
+      return MOE_ERR_CUDA;
+    g_no_alloc_ptr[dev] = ptr;
+  }
+  *out = g_no_alloc_ptr[dev];
+  return MOE_OK;
+}
+
 // bf16 tensor map over a row-major [outer][mid][inner] array (mid = 1 for 2D),
 // 128-byte swizzle, box {64, box_rows(, 1)}; out-of-range rows read as zero.
 bool encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
@@ -606,8 +629,27 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_SCRATCH_LIMIT: return "MOE_ERR_SCRATCH_LIMIT";
   }
   return "MOE_STATUS_UNKNOWN";
+}
+
+moe_status moe_forward_no_alloc(const moe_dims* dims, const void* x, const float* W_r,
+                                const void* W_g, const void* W_u, const void* W_d,
+                                const void* W_shared, int E, int k, float capacity_factor,
+                                void* y, float* aux, int32_t* counts) {
+  const moe_status s = check_dims(dims, E, k, capacity_factor);
+  if (s != MOE_OK) return s;
+  if (make_plan(dims, E, k, capacity_factor).total > MOE_NO_ALLOC_WORKSPACE_BYTES)
+    return MOE_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  const moe_status ss = no_alloc_scratch(&scratch);
+  if (ss != MOE_OK) return ss;
+  moe_dims d2 = *dims;
+  d2.workspace = scratch;
+  d2.workspace_bytes = MOE_NO_ALLOC_WORKSPACE_BYTES;
+  return forward_impl(&d2, x, W_r, W_g, W_u, W_d, W_shared, E, k, capacity_factor, y, aux,
+                      counts);
 }
 
 }  // extern "C"
