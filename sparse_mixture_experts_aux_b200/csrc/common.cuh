@@ -15,8 +15,9 @@ constexpr int DEVERR_TIMEOUT = 1;
 // this many rows, so that no GEMM M-tile straddles two experts.
 constexpr int ROW_TILE = 128;
 
-// Tokens handled by one block of the routing kernel (8 warps x 32 tokens).
-constexpr int ROUTE_CHUNK = 256;
+// Tokens handled by one block of the routing kernel (8 warps x 8 tokens); the
+// stable ranks are counted per chunk, so this is also the rank-base granule.
+constexpr int ROUTE_CHUNK = 64;
 constexpr int ROUTE_WARPS = 8;
 
 __device__ __forceinline__ float to_f32(float v) { return v; }

@@ -83,8 +83,9 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
     return o;
   };
   const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
-  p.router_narrow = E <= 16 && p.T >= 1024;
-  p.router_split = p.router_narrow ? 1 : moe::simt_split_k(p.T, E, p.d);
+  p.router_narrow = E <= 16;
+  p.router_split = p.router_narrow ? moe::narrow_split_k(p.T, E, p.d)
+                                   : moe::simt_split_k(p.T, E, p.d);
   p.o_logits = take(static_cast<size_t>(p.router_split) * T * E * 4);
   p.o_idx = take(TK * 4);
   p.o_gate = take(TK * 4);
@@ -92,7 +93,7 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   p.o_slot = take(TK * 4);
   p.o_hist = take(static_cast<size_t>(p.nblk) * E * 4);
   p.o_base = take(static_cast<size_t>(p.nblk) * E * 4);
-  p.o_psum_part = take(static_cast<size_t>(p.nblk) * moe::ROUTE_WARPS * E * 8);
+  p.o_psum_part = take(static_cast<size_t>(p.nblk) * E * 8);
   p.o_probsum = take(static_cast<size_t>(E) * 8);
   p.o_tile_start = take(static_cast<size_t>(E + 1) * 4);
   p.o_pair_start = take(static_cast<size_t>(E + 1) * 4);
@@ -180,7 +181,7 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
         !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
       return MOE_ERR_CUDA;
-    const int rs = 2 * moe::ROUTE_WARPS * moe::tc::MAX_E * 4;
+    const int rs = static_cast<int>(moe::route_smem_bytes(moe::tc::MAX_E));
     if (cudaFuncSetAttribute(moe::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              rs) != cudaSuccess ||
         cudaFuncSetAttribute(moe::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -280,12 +281,15 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   moe::SimtGroup none{};
   tm.at(0);
   if (P.router_narrow) {
-    const int warps = (T + moe::ROUTER_TOK - 1) / moe::ROUTER_TOK;
-    const int blocks = (warps + 7) / 8;
-    if (P.E <= 8)
-      moe::router_narrow_kernel<TX, 1><<<blocks, 256, 0, st>>>(x, W_r, T, P.d, P.E, logits);
-    else
-      moe::router_narrow_kernel<TX, 2><<<blocks, 256, 0, st>>>(x, W_r, T, P.d, P.E, logits);
+    if (P.E <= 8) {
+      dim3 grid((T + moe::NarrowShape<8>::TB - 1) / moe::NarrowShape<8>::TB, P.router_split);
+      moe::router_narrow_kernel<TX, 8>
+          <<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split, logits);
+    } else {
+      dim3 grid((T + moe::NarrowShape<16>::TB - 1) / moe::NarrowShape<16>::TB, P.router_split);
+      moe::router_narrow_kernel<TX, 16>
+          <<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split, logits);
+    }
   } else {
     dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM,
               P.router_split);
@@ -297,7 +301,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   // (1) routing
   tm.at(2);
   {
-    const size_t smem = static_cast<size_t>(2) * moe::ROUTE_WARPS * P.E * 4;
+    const size_t smem = moe::route_smem_bytes(P.E);
     const int nv = (P.E + 31) / 32;
 #define MOE_ROUTE(NV)                                                                           \
   moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(logits, P.router_split, dims->router_bias, \
@@ -316,7 +320,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
 
   // (2) scan: counts, capacity, segment offsets, aux
   tm.at(4);
-  moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk * moe::ROUTE_WARPS, P.E,
+  moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk, P.E,
                                        P.T, P.k, P.C, counts, base, tile_start, pair_start,
                                        probsum, aux);
   tm.at(5);
@@ -324,8 +328,12 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
 
   // (3) scatter rows into expert segments
   tm.at(6);
-  moe::scatter_kernel<TX><<<(T + 7) / 8, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
-                                                       base, tile_start, slot, rowgate, xp);
+  {
+    const int nvec = static_cast<int>(static_cast<size_t>(P.d) * sizeof(TX) / 16);
+    dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
+    moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
+                                                  base, tile_start, slot, rowgate, xp);
+  }
   tm.at(7);
   return launched();
 }
@@ -491,8 +499,12 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     }
     // (6) combine
     tm.at(12);
-    moe::combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
-                                                           static_cast<bf16*>(y));
+    {
+      const int nvec = P.d * 2 / 16;
+      dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
+      moe::combine_kernel<bf16><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+                                                      static_cast<bf16*>(y));
+    }
     tm.at(13);
     return launched();
   }
@@ -535,8 +547,12 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
   }
   tm.at(12);
-  moe::combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
-                                                          static_cast<float*>(y));
+  {
+    const int nvec = P.d * 4 / 16;
+    dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
+    moe::combine_kernel<float><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+                                                     static_cast<float*>(y));
+  }
   tm.at(13);
   return launched();
 }

@@ -13,11 +13,18 @@
 
 namespace moe {
 
-// One warp per token. Lane s (< k) resolves assignment s: its rank in token
-// order within the expert is base[chunk][e] + lrank; it is kept when the rank
-// is below the capacity C, and lands at row tile_start[e]*ROW_TILE + rank.
-// The token's row is then copied to every kept position with 16-byte loads
-// and stores (coalesced across the warp).
+// Column chunk of one warp in the scatter and combine kernels: 32 lanes x
+// PERMUTE_VPL 16-byte vectors. grid.y walks the chunks of a row, so a small
+// batch still spreads over many SMs.
+constexpr int PERMUTE_VPL = 4;
+constexpr int PERMUTE_CHUNK_VECS = 32 * PERMUTE_VPL;
+
+// One warp per (token, column chunk). Lane s (< k) resolves assignment s: its
+// rank in token order within the expert is base[chunk][e] + lrank; it is kept
+// when the rank is below the capacity C, and lands at row
+// tile_start[e]*ROW_TILE + rank (blocks with blockIdx.y == 0 record it). The
+// chunk of the token's row is then copied to every kept position with 16-byte
+// loads and stores (coalesced across the warp).
 template <typename TX>
 __global__ void __launch_bounds__(256) scatter_kernel(
     const TX* __restrict__ x, int d, int T, int k, int E, int64_t C,
@@ -33,25 +40,28 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const size_t a = (size_t)t * k + lane;
     const int e = idx[a];
     const int rank = base[(size_t)(t / ROUTE_CHUNK) * E + e] + lrank[a];
-    if (C < 0 || (int64_t)rank < C) {
-      mypos = tile_start[e] * ROW_TILE + rank;
-      row_gate[mypos] = gate[a];
+    if (C < 0 || (int64_t)rank < C) mypos = tile_start[e] * ROW_TILE + rank;
+    if (blockIdx.y == 0) {
+      if (mypos >= 0) row_gate[mypos] = gate[a];
+      slot_pos[a] = mypos;
     }
-    slot_pos[a] = mypos;
   }
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   const int nvec = (int)((size_t)d * sizeof(TX) / 16);
+  const int c_begin = blockIdx.y * PERMUTE_CHUNK_VECS;
+  const int c_end = c_begin + PERMUTE_CHUNK_VECS < nvec ? c_begin + PERMUTE_CHUNK_VECS : nvec;
   for (int s = 0; s < k; ++s) {
     const int p = __shfl_sync(0xffffffffu, mypos, s);
     if (p < 0) continue;
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)p * d);
-    for (int c = lane; c < nvec; c += 32) st_v4(dst + c, ld_nc_v4(src + c));
+    for (int c = c_begin + lane; c < c_end; c += 32) st_v4(dst + c, ld_nc_v4(src + c));
   }
 }
 
-// One warp per token: y[t] = sum_s Yrows[slot_pos[t][s]] (dropped slots skipped)
-// + Ys[t] (shared expert, if any), summed in fp32 in slot order with a single
-// rounding to the output type. Yrows already carry the gate factor.
+// One warp per (token, column chunk): y[t] = sum_s Yrows[slot_pos[t][s]]
+// (dropped slots skipped) + Ys[t] (shared expert, if any), summed in fp32 in
+// slot order with a single rounding to the output type. Yrows already carry
+// the gate factor.
 template <typename TY>
 __global__ void __launch_bounds__(256) combine_kernel(
     const TY* __restrict__ yrows, const TY* __restrict__ ys, const int32_t* __restrict__ slot_pos,
@@ -62,9 +72,11 @@ __global__ void __launch_bounds__(256) combine_kernel(
   if (t >= T) return;  // warp-uniform
   const int mypos = (lane < k) ? slot_pos[(size_t)t * k + lane] : -1;
   const int nvec = (int)((size_t)d * sizeof(TY) / 16);
-  for (int c0 = 0; c0 < nvec; c0 += 32) {
+  const int c_begin = blockIdx.y * PERMUTE_CHUNK_VECS;
+  const int c_end = c_begin + PERMUTE_CHUNK_VECS < nvec ? c_begin + PERMUTE_CHUNK_VECS : nvec;
+  for (int c0 = c_begin; c0 < c_end; c0 += 32) {
     const int c = c0 + lane;
-    const bool active = c < nvec;
+    const bool active = c < c_end;
     float acc[VN];
 #pragma unroll
     for (int i = 0; i < VN; ++i) acc[i] = 0.f;

@@ -202,16 +202,17 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
 }
 
 // ---------------------------------------------------------------------------
-// Router logits for few experts (E <= 8 * NG): r[t, e] = sum_j x[t, j] W_r[e, j].
-// Memory-bound on x, so there is no output tile to waste: each warp owns
-// ROUTER_TOK consecutive tokens over the whole of K; lane l takes the 8
-// consecutive elements at 8l + 256i of every row, multiplies them by the same
-// slice of every router row (read through L1, shared by all warps), and keeps
-// one fp32 partial per (token, expert). The 32 lane partials of each output
-// are then summed by a fixed butterfly, so the result is deterministic. Each
-// lane's chain has d/32 terms.
+// Router logits for few experts (E <= NE, NE = 8 or 16): r[t, e] = sum_j x[t, j] W_r[e, j].
+// This is bound by reading x, so there is no wasted output tile. A block
+// owns NARROW_TB tokens and one K range (grid.y splits K; the routing kernel
+// sums the split partials in a fixed order). Router rows are staged in shared
+// memory 256 columns at a time and read by all 8 warps. Warp w owns tokens
+// w*TOK .. w*TOK+TOK-1, and lane l takes columns 8l..8l+7 of each chunk.
+// Every (token, expert) keeps one fp32 partial per lane: a chunk adds a dot
+// of 8 terms to it (blocked summation), and the 32 lane partials are then
+// summed by a fixed butterfly. The result is deterministic.
 // ---------------------------------------------------------------------------
-constexpr int ROUTER_TOK = 4;
+constexpr int NARROW_KC = 256;  // columns per staged chunk
 
 template <typename TA>
 __device__ __forceinline__ void load8(const TA* p, float* f);
@@ -225,71 +226,105 @@ __device__ __forceinline__ void load8<float>(const float* p, float* f) {
   Vec16<float>::unpack(ld_nc_v4(p + 4), f + 4);
 }
 
-template <typename TA, int NG>  // NG groups of 8 experts
+template <int NE> struct NarrowShape {
+  static constexpr int TOK = NE <= 8 ? 8 : 4;  // tokens per warp
+  static constexpr int TB = 8 * TOK;           // tokens per block
+};
+
+// K chunks for the narrow router: enough blocks for about two waves.
+inline int narrow_split_k(int64_t T, int E, int d) {
+  const int tb = E <= 8 ? NarrowShape<8>::TB : NarrowShape<16>::TB;
+  const int64_t blocks = (T + tb - 1) / tb;
+  const int chunks = d / NARROW_KC > 0 ? d / NARROW_KC : 1;
+  int split = 1;
+  while (blocks * split < 296 && split * 2 <= chunks) split *= 2;
+  return split;
+}
+
+template <typename TA, int NE>
 __global__ void __launch_bounds__(256) router_narrow_kernel(const TA* __restrict__ x,
                                                             const float* __restrict__ W_r, int T,
-                                                            int d, int E,
+                                                            int d, int E, int splits,
                                                             float* __restrict__ logits) {
+  constexpr int TOK = NarrowShape<NE>::TOK;
+  constexpr int TB = NarrowShape<NE>::TB;
+  __shared__ __align__(16) float ws[NE][NARROW_KC];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = (blockIdx.x * (blockDim.x >> 5) + warp) * ROUTER_TOK;
-  if (t0 >= T) return;  // warp-uniform
-  float acc[ROUTER_TOK][NG * 8];
+  const int t0 = blockIdx.x * TB + warp * TOK;
+  // K range of this split: whole chunks, the last split takes the remainder
+  const int chunks = (d + NARROW_KC - 1) / NARROW_KC;
+  const int per = (chunks + splits - 1) / splits;
+  const int c_begin = blockIdx.y * per;
+  const int c_end = c_begin + per < chunks ? c_begin + per : chunks;
+  float acc[TOK][NE];
 #pragma unroll
-  for (int t = 0; t < ROUTER_TOK; ++t)
+  for (int t = 0; t < TOK; ++t)
 #pragma unroll
-    for (int e = 0; e < NG * 8; ++e) acc[t][e] = 0.f;
-  for (int j = lane * 8; j < d; j += 256) {
-    float xv[ROUTER_TOK][8];
+    for (int e = 0; e < NE; ++e) acc[t][e] = 0.f;
+  for (int c = c_begin; c < c_end; ++c) {
+    const int k0 = c * NARROW_KC;
+    const int kw = d - k0 < NARROW_KC ? d - k0 : NARROW_KC;  // a multiple of 8
+    __syncthreads();  // previous chunk fully consumed
+    for (int i = threadIdx.x; i < NE * (NARROW_KC / 4); i += blockDim.x) {
+      const int e = i / (NARROW_KC / 4), q = (i % (NARROW_KC / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E && q < kw) v = *reinterpret_cast<const float4*>(W_r + (size_t)e * d + k0 + q);
+      *reinterpret_cast<float4*>(&ws[e][q]) = v;
+    }
+    const int j = lane * 8;
+    float xv[TOK][8];
 #pragma unroll
-    for (int t = 0; t < ROUTER_TOK; ++t) {
-      if (t0 + t < T) load8<TA>(x + (size_t)(t0 + t) * d + j, xv[t]);
+    for (int t = 0; t < TOK; ++t) {
+      if (t0 + t < T && j < kw) load8<TA>(x + (size_t)(t0 + t) * d + k0 + j, xv[t]);
       else
 #pragma unroll
         for (int i = 0; i < 8; ++i) xv[t][i] = 0.f;
     }
+    __syncthreads();
 #pragma unroll
-    for (int e = 0; e < NG * 8; ++e) {
-      if (e < E) {
-        float wv[8];
-        load8<float>(W_r + (size_t)e * d + j, wv);
+    for (int e = 0; e < NE; ++e) {
+      const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][j]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&ws[e][j + 4]);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int t = 0; t < ROUTER_TOK; ++t) {
-          float part = 0.f;
+      for (int t = 0; t < TOK; ++t) {
+        float part = 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) part = fmaf(xv[t][i], wv[i], part);
-          acc[t][e] += part;
-        }
+        for (int i = 0; i < 8; ++i) part = fmaf(xv[t][i], wv[i], part);
+        acc[t][e] += part;
       }
     }
   }
 #pragma unroll
-  for (int t = 0; t < ROUTER_TOK; ++t)
+  for (int t = 0; t < TOK; ++t)
 #pragma unroll
-    for (int e = 0; e < NG * 8; ++e) {
+    for (int e = 0; e < NE; ++e) {
       float v = acc[t][e];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       acc[t][e] = v;
     }
-  if (lane == 0) {
+  // lane (t * NE + e) % 32 writes output (t, e)
+  float* out = logits + (size_t)blockIdx.y * T * E;
 #pragma unroll
-    for (int t = 0; t < ROUTER_TOK; ++t)
-      if (t0 + t < T)
+  for (int t = 0; t < TOK; ++t)
 #pragma unroll
-        for (int e = 0; e < NG * 8; ++e)
-          if (e < E) logits[(size_t)(t0 + t) * E + e] = acc[t][e];
-  }
+    for (int e = 0; e < NE; ++e)
+      if (lane == ((t * NE + e) & 31) && e < E && t0 + t < T)
+        out[(size_t)(t0 + t) * E + e] = acc[t][e];
 }
 
 // ---------------------------------------------------------------------------
-// Routing: one warp per token, ROUTE_CHUNK tokens per block.
+// Routing: ROUTE_CHUNK tokens per block, ROUTE_WARPS warps, each warp owning
+// ROUTE_CHUNK / ROUTE_WARPS consecutive tokens, one token at a time:
 //   softmax over all E logits (+ optional bias), per-expert probability sums
 //   accumulated in fp64 in a fixed order; top-k by k rounds of a warp argmax
 //   ordered by (logit descending, index ascending); gates as a softmax over
-//   the k kept logits; then stable ranks: for each assignment, how many
+//   the k kept logits. Then stable ranks: for each assignment, how many
 //   earlier tokens of the same chunk chose the same expert (a 32-bit token
-//   mask per warp and expert, prefix-summed over the chunk's warps).
-// Outputs per block: hist[blk][e] and per-warp probability-sum partials.
+//   mask per 32-token group and expert, prefix-summed over the groups).
+// Outputs per block: hist[blk][e] and the block's probability sums (the
+// warps' fp64 partials added in warp order).
 // NV = ceil(E / 32) logits held per lane.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_max(float v) {
@@ -303,20 +338,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+constexpr int ROUTE_TOK_PER_WARP = ROUTE_CHUNK / ROUTE_WARPS;
+constexpr int ROUTE_RANK_GROUPS = ROUTE_CHUNK / 32;
+static_assert(ROUTE_CHUNK % 32 == 0 && ROUTE_RANK_GROUPS <= ROUTE_WARPS, "route chunk shape");
+
+// Dynamic shared memory of route_kernel for E experts.
+__host__ __device__ constexpr size_t route_smem_bytes(int E) {
+  return (size_t)ROUTE_WARPS * E * 8 + (size_t)2 * ROUTE_RANK_GROUPS * E * 4;
+}
+
 template <int NV>
 __global__ void __launch_bounds__(256) route_kernel(
     float* __restrict__ logits, int splits, const float* __restrict__ bias, int T, int E, int k,
     int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int32_t* __restrict__ lrank_out,
     int32_t* __restrict__ hist, double* __restrict__ psum_part) {
-  extern __shared__ uint32_t route_smem[];
-  uint32_t* bm = route_smem;                                   // [ROUTE_WARPS][E] token masks
-  int32_t* wbase = reinterpret_cast<int32_t*>(route_smem + ROUTE_WARPS * E);  // [ROUTE_WARPS][E]
+  extern __shared__ __align__(16) uint8_t route_smem_raw[];
+  double* red = reinterpret_cast<double*>(route_smem_raw);  // [ROUTE_WARPS][E]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(red + (size_t)ROUTE_WARPS * E);  // [groups][E]
+  int32_t* wbase = reinterpret_cast<int32_t*>(bm + (size_t)ROUTE_RANK_GROUPS * E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blk = blockIdx.x;
-  for (int i = threadIdx.x; i < ROUTE_WARPS * E; i += blockDim.x) bm[i] = 0u;
-  __syncthreads();
+  for (int i = threadIdx.x; i < ROUTE_RANK_GROUPS * E; i += blockDim.x) bm[i] = 0u;
 
-  const int t_warp0 = blk * ROUTE_CHUNK + warp * 32;
+  const int t_warp0 = blk * ROUTE_CHUNK + warp * ROUTE_TOK_PER_WARP;
   double ps[NV];
   float bv[NV];
 #pragma unroll
@@ -344,13 +388,13 @@ __global__ void __launch_bounds__(256) route_kernel(
     }
   };
   if (t_warp0 < T) load_logits(t_warp0);
-  for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < ROUTE_TOK_PER_WARP; ++j) {
     const int t = t_warp0 + j;
     if (t >= T) break;  // warp-uniform
     float raw[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) raw[i] = nxt[i];
-    if (j + 1 < 32 && t + 1 < T) load_logits(t + 1);
+    if (j + 1 < ROUTE_TOK_PER_WARP && t + 1 < T) load_logits(t + 1);
     float* row = logits + (size_t)t * E;
     float v[NV];
     uint32_t removed = 0u;
@@ -409,32 +453,39 @@ __global__ void __launch_bounds__(256) route_kernel(
       gate_out[(size_t)t * k + lane] = z / zs;
     }
   }
-  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) red[(size_t)warp * E + e] = ps[i];
+  }
+  __syncthreads();  // every token's choices are in idx_out, every partial in red
 
-  const int t = t_warp0 + lane;
-  if (t < T) {
+  const int t = blk * ROUTE_CHUNK + warp * 32 + lane;  // rank phase: warps 0..groups-1
+  const bool ranker = warp < ROUTE_RANK_GROUPS && t < T;
+  if (ranker) {
     for (int sl = 0; sl < k; ++sl) {
       const int e = idx_out[(size_t)t * k + sl];
       atomicOr(&bm[warp * E + e], 1u << lane);
     }
   }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    double acc = 0.0;
+#pragma unroll
+    for (int w = 0; w < ROUTE_WARPS; ++w) acc += red[(size_t)w * E + e];  // fixed order
+    psum_part[(size_t)blk * E + e] = acc;
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
 #pragma unroll
-    for (int w = 0; w < ROUTE_WARPS; ++w) {
-      wbase[w * E + e] = run;
-      run += __popc(bm[w * E + e]);
+    for (int g = 0; g < ROUTE_RANK_GROUPS; ++g) {
+      wbase[g * E + e] = run;
+      run += __popc(bm[g * E + e]);
     }
     hist[(size_t)blk * E + e] = run;
   }
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) psum_part[((size_t)blk * ROUTE_WARPS + warp) * E + e] = ps[i];
-  }
   __syncthreads();
-  if (t < T) {
+  if (ranker) {
     const uint32_t lt = (1u << lane) - 1u;
     for (int sl = 0; sl < k; ++sl) {
       const int e = idx_out[(size_t)t * k + sl];
@@ -465,6 +516,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(
   double term = 0.0;
   if (e < E) {
     int run = 0;
+#pragma unroll 8
     for (int b = 0; b < nblk; ++b) {
       base[(size_t)b * E + e] = run;
       run += hist[(size_t)b * E + e];
@@ -473,6 +525,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(
     const int kept = (C >= 0 && (int64_t)run > C) ? (int)C : run;
     tiles = (kept + ROW_TILE - 1) / ROW_TILE;
     double ps = 0.0;
+#pragma unroll 8
     for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
     probsum[e] = ps;
     term = (double)run * ps;
