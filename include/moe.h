@@ -74,7 +74,34 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 #define MOE_NUM_KERNELS 7
 
 /* Limits of this build: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
- * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1). */
+ * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1);
+ * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group. */
+
+/*
+ * Routing variants (gate_mode, selection_bias, n_group / topk_group).
+ *   MOE_GATE_RENORM  g = softmax over the chosen logits (the definition above).
+ *   MOE_GATE_RAW     g_i = p_i, the softmax over all experts, not renormalised:
+ *                    Switch's top-1 form (jacopoparretti "Mixture of experts,
+ *                    token by token", "Experts and a router"; kevinluzbetak
+ *                    routing example, "some implementations skip the
+ *                    renormalisation").
+ *   MOE_GATE_SIGMOID affinities s_i = sigmoid(r_i), top-k on s, g = s_K / sum s_K
+ *                    (DeepSeek-V3: AI Engineering Illustrated "Mixture of
+ *                    Experts", "The router is small but it decides everything").
+ *                    Here P_i of the balance statistic is the mean of
+ *                    s_i / sum_j s_j over all experts.
+ * selection_bias: added to the logit (RENORM, RAW) or to the affinity
+ * (SIGMOID) only when choosing the experts; the gates ignore it (DeepSeek-V3's
+ * balancing bias: AI Engineering Illustrated, "Fix 2 nudges a bias instead";
+ * jacopoparretti, "A bias").
+ * Group-limited selection (jacopoparretti, "Smaller experts, more of them": 4 of
+ * 8 groups): a group's score is its largest selection score; a token keeps the
+ * topk_group best groups (ties to the lower group) and picks its k experts
+ * among them.
+ */
+#define MOE_GATE_RENORM 0
+#define MOE_GATE_RAW 1
+#define MOE_GATE_SIGMOID 2
 
 typedef struct {
   int64_t T;                 /* tokens in this call (0 allowed: empty batch) */
@@ -82,7 +109,8 @@ typedef struct {
   int32_t d_e;               /* routed expert hidden width */
   int32_t d_s;               /* shared expert hidden width; 0 = no shared expert */
   int32_t dtype;             /* moe_dtype of x, W_g, W_u, W_d, W_shared and y */
-  int32_t gate_mode;         /* 0 = renormalised top-k gates (only value accepted) */
+  int32_t gate_mode;         /* MOE_GATE_RENORM (0), MOE_GATE_RAW (1) or MOE_GATE_SIGMOID (2),
+                                see "Routing variants" above */
   const float* router_bias;  /* device [E] fp32 added to the logits before softmax
                                 and top-k, or NULL */
   void* workspace;           /* device scratch of >= moe_workspace_size() bytes,
@@ -92,6 +120,11 @@ typedef struct {
   void* const* events;       /* optional cudaEvent_t[2*MOE_NUM_KERNELS]; when non-NULL,
                                 events[2i] / events[2i+1] are recorded on `stream`
                                 right before / after kernel i (NULL entries skipped) */
+  const float* selection_bias; /* device [E] fp32 added to the selection scores only
+                                  (who is picked, not the gates), or NULL */
+  int32_t n_group;           /* group-limited selection: experts form n_group contiguous
+                                groups of E / n_group; 0 or 1 = no groups */
+  int32_t topk_group;        /* groups a token may pick from (1 <= topk_group <= n_group) */
   uint64_t wait_timeout_ns;  /* limit of each device-side mbarrier wait in the GEMM
                                 kernels; 0 = default (4 s). A tiny value makes the waits
                                 expire on purpose: the kernels then record

@@ -50,6 +50,8 @@ import numpy as np
 __all__ = [
     "router_logits", "softmax_all", "top_k", "gates_softmax_topk", "gates_renormalised",
     "topk_margin", "capacity_limit", "capacity_keep", "silu", "swiglu_ffn",
+    "GATE_RENORM", "GATE_RAW", "GATE_SIGMOID", "sigmoid_affinity", "balance_probs",
+    "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
     "moe_param_count", "active_flops", "OracleResult",
 ]
@@ -121,6 +123,98 @@ def topk_margin(r: np.ndarray, k: int) -> np.ndarray:
         return np.full(r.shape[0], np.inf)
     s = -np.sort(-r, axis=1)
     return s[:, k - 1] - s[:, k]
+
+
+# ----------------------------------------------------------------------------
+# Gate variants and DeepSeek-V3 scoring
+#   mode 1, raw softmax gates: [JP] "Experts and a router" (Switch takes a
+#     softmax over all experts first and keeps only the top one); [KL] routing
+#     worked example (some implementations skip the renormalisation).
+#   selection-only bias: [AEI] "Fix 2 nudges a bias instead" and [JP] "A bias"
+#     (a per-expert bias added to the score only when picking the top k; the
+#     mixing weights ignore it).
+#   mode 2, sigmoid affinities: [AEI] "The router is small but it decides
+#     everything" and [JP] "Experts and a router" (a sigmoid per expert, top k,
+#     then the k chosen affinities normalised to sum to one).
+#   group-limited selection: [JP] "Smaller experts, more of them" (each token
+#     is limited to 4 of its 8 expert groups; the released configuration has
+#     n_group 8, topk_group 4).
+# Readings where the pages are silent:
+#   R7  the raw-probability gates of mode 1 are not renormalised for any k;
+#   R8  in mode 2, P_i of the balance statistic is the mean over tokens of the
+#       affinity normalised over all experts, s_i / sum_j s_j;
+#   R9  groups are contiguous blocks of E / n_group experts; a group's score is
+#       its largest selection score; equal group scores go to the lower group;
+#   R10 the selection bias is added to the logit (modes 0, 1) or to the
+#       affinity (mode 2); the router bias of R6 still enters before everything.
+# ----------------------------------------------------------------------------
+GATE_RENORM, GATE_RAW, GATE_SIGMOID = 0, 1, 2
+
+
+def sigmoid_affinity(r: np.ndarray) -> np.ndarray:
+    """s = 1 / (1 + e^{-r}), elementwise."""
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-r))
+
+
+def balance_probs(r: np.ndarray, gate_mode: int) -> np.ndarray:
+    """Per-token, per-expert probabilities whose mean is P_i (R4, R8)."""
+    if gate_mode == GATE_SIGMOID:
+        s = sigmoid_affinity(r)
+        return s / s.sum(axis=1, keepdims=True)
+    return softmax_all(r)
+
+
+def selection_scores(r: np.ndarray, gate_mode: int, selection_bias=None) -> np.ndarray:
+    """What the top-k ranks: the logit (modes 0, 1) or the affinity (mode 2),
+    plus the selection-only bias (R10)."""
+    sel = sigmoid_affinity(r) if gate_mode == GATE_SIGMOID else r.copy()
+    if selection_bias is not None:
+        sel = sel + _f64(selection_bias)[None, :]
+    return sel
+
+
+def group_eligible(sel: np.ndarray, n_group: int, topk_group: int):
+    """Experts a token may pick under group-limited routing (R9), and the gap
+    between the topk_group-th and the next group score (+inf if all kept)."""
+    T, E = sel.shape
+    if n_group <= 1 or topk_group >= n_group:
+        return np.ones((T, E), dtype=bool), np.full(T, np.inf)
+    gsize = E // n_group
+    gscore = sel.reshape(T, n_group, gsize).max(axis=2)
+    order = np.argsort(-gscore, axis=1, kind="stable")
+    keep_groups = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(keep_groups, order[:, :topk_group], True, axis=1)
+    srt = np.take_along_axis(gscore, order, axis=1)
+    return np.repeat(keep_groups, gsize, axis=1), srt[:, topk_group - 1] - srt[:, topk_group]
+
+
+def select_experts(sel: np.ndarray, k: int, eligible: np.ndarray):
+    """Top-k of the selection scores among eligible experts (ties to the lower
+    index), in slot order, and the k-th/(k+1)-th gap among the eligible."""
+    masked = np.where(eligible, sel, -np.inf)
+    order = np.argsort(-masked, axis=1, kind="stable")
+    idx = order[:, :k].astype(np.int64)
+    srt = np.take_along_axis(masked, order, axis=1)
+    if k < sel.shape[1]:
+        nxt = srt[:, k]
+        gap = np.where(np.isfinite(nxt), srt[:, k - 1] - nxt, np.inf)
+    else:
+        gap = np.full(sel.shape[0], np.inf)
+    return idx, gap
+
+
+def gates_for_mode(r: np.ndarray, idx: np.ndarray, gate_mode: int) -> np.ndarray:
+    """Mixing weights of the chosen experts, from the logits without the
+    selection bias: mode 0 softmax over the chosen logits ([ZTF] "The MoE
+    layer"); mode 1 the raw softmax probabilities (R7); mode 2 the chosen
+    sigmoid affinities normalised to sum to one."""
+    if gate_mode == GATE_RAW:
+        return np.take_along_axis(softmax_all(r), idx, axis=1)
+    if gate_mode == GATE_SIGMOID:
+        sk = np.take_along_axis(sigmoid_affinity(r), idx, axis=1)
+        return sk / sk.sum(axis=1, keepdims=True)
+    return gates_softmax_topk(r, idx)
 
 
 # ----------------------------------------------------------------------------
@@ -213,7 +307,8 @@ class OracleResult:
 def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
                 capacity_factor: float = 0.0, router_bias=None,
                 shared_weights: Optional[Sequence] = None,
-                rows: Optional[np.ndarray] = None) -> OracleResult:
+                rows: Optional[np.ndarray] = None, gate_mode: int = GATE_RENORM,
+                selection_bias=None, n_group: int = 1, topk_group: int = 1) -> OracleResult:
     """Forward pass of the routed MoE FFN layer, looping over experts.
 
     x: [T, d]; W_r: [E, d]; expert_weights(e) -> (W_g[e], W_u[e], W_d[e]);
@@ -226,13 +321,22 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
     gates; counts; capacity cut in token order; then for each expert, its kept
     tokens in one batch through the SwiGLU, scaled by the gate and added into y;
     the shared expert on every token with weight 1; the balance statistic.
+    gate_mode, selection_bias, n_group and topk_group select the routing
+    variants above (defaults: renormalised softmax top-k, no bias, no groups).
     """
     T = x.shape[0]
     r = router_logits(x, W_r, router_bias)
     E = r.shape[1]
-    p = softmax_all(r)
-    idx = top_k(r, k)
-    g = gates_softmax_topk(r, idx)
+    p = balance_probs(r, gate_mode)
+    if gate_mode == GATE_RENORM and selection_bias is None and n_group <= 1:
+        idx = top_k(r, k)
+        margin = topk_margin(r, k)
+    else:
+        sel = selection_scores(r, gate_mode, selection_bias)
+        eligible, gmargin = group_eligible(sel, n_group, topk_group)
+        idx, kmargin = select_experts(sel, k, eligible)
+        margin = np.minimum(kmargin, gmargin)
+    g = gates_for_mode(r, idx, gate_mode)
     counts = np.bincount(idx.ravel(), minlength=E).astype(np.int64)
     C = capacity_limit(capacity_factor, T, k, E)
     keep = capacity_keep(idx, E, C)
@@ -258,7 +362,7 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
 
     return OracleResult(logits=r, probs=p, idx=idx, gates=g, counts=counts,
                         capacity=C, keep=keep, probsum=probsum, aux=aux,
-                        margin=topk_margin(r, k), rows=rows, y=y[rows],
+                        margin=margin, rows=rows, y=y[rows],
                         dropped_fraction=dropped_fraction(counts, C, T, k))
 
 

@@ -21,6 +21,7 @@ MOE_ERR_SCRATCH_LIMIT = 6
 MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
+MOE_GATE_RENORM, MOE_GATE_RAW, MOE_GATE_SIGMOID = 0, 1, 2
 MOE_NUM_KERNELS = 7
 KERNEL_NAMES = ("router_logits", "route", "scan", "scatter", "gate_up_swiglu", "down_scale", "combine")
 
@@ -42,6 +43,9 @@ class moe_dims(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
         ("events", ctypes.c_void_p),
+        ("selection_bias", ctypes.c_void_p),
+        ("n_group", ctypes.c_int32),
+        ("topk_group", ctypes.c_int32),
         ("wait_timeout_ns", ctypes.c_uint64),
     ]
 
@@ -122,7 +126,8 @@ def _ptr(t) -> int:
 
 def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, router_bias=None,
               workspace=None, workspace_bytes: int = 0, stream: int = 0, events=None,
-              gate_mode: int = 0, wait_timeout_ns: int = 0) -> moe_dims:
+              gate_mode: int = 0, wait_timeout_ns: int = 0, selection_bias=None,
+              n_group: int = 0, topk_group: int = 0) -> moe_dims:
     """Fill a moe_dims. `events` is a ctypes array of cudaEvent_t handles or None."""
     dims = moe_dims()
     dims.T, dims.d, dims.d_e, dims.d_s = int(T), int(d), int(d_e), int(d_s)
@@ -133,6 +138,8 @@ def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, rou
     dims.stream = int(stream) or None
     dims.events = ctypes.cast(events, ctypes.c_void_p) if events is not None else None
     dims.wait_timeout_ns = int(wait_timeout_ns)
+    dims.selection_bias = _ptr(selection_bias) or None
+    dims.n_group, dims.topk_group = int(n_group), int(topk_group)
     return dims
 
 

@@ -52,8 +52,17 @@ moe_status check_dims(const moe_dims* dims, int E, int k, float cf) {
   if (dims->dtype != MOE_F32 && dims->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (isnan(cf)) return MOE_ERR_INVALID_ARG;
-  if (dims->gate_mode != 0) return MOE_ERR_UNSUPPORTED;
+  if (dims->gate_mode < MOE_GATE_RENORM || dims->gate_mode > MOE_GATE_SIGMOID)
+    return MOE_ERR_INVALID_ARG;
   if (E > moe::tc::MAX_E || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (dims->n_group > 1) {
+    if (dims->n_group > 32) return MOE_ERR_UNSUPPORTED;
+    if (E % dims->n_group != 0 || dims->topk_group < 1 || dims->topk_group > dims->n_group ||
+        static_cast<int64_t>(k) > static_cast<int64_t>(dims->topk_group) * (E / dims->n_group))
+      return MOE_ERR_INVALID_ARG;
+  } else if (dims->n_group < 0) {
+    return MOE_ERR_INVALID_ARG;
+  }
   if (dims->T * static_cast<int64_t>(k) >= (int64_t(1) << 31) ||
       dims->T * static_cast<int64_t>(E) >= (int64_t(1) << 40))
     return MOE_ERR_UNSUPPORTED;
@@ -304,8 +313,9 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
     const size_t smem = moe::route_smem_bytes(P.E);
     const int nv = (P.E + 31) / 32;
 #define MOE_ROUTE(NV)                                                                           \
-  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(logits, P.router_split, dims->router_bias, \
-                                                   T, P.E, P.k, idx, \
+  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(                                         \
+      logits, P.router_split, dims->router_bias, dims->selection_bias, dims->gate_mode,         \
+      dims->n_group, dims->topk_group, T, P.E, P.k, idx, \
                                                    gate, lrank, hist, psum_part)
     if (nv <= 1) MOE_ROUTE(1);
     else if (nv <= 2) MOE_ROUTE(2);
@@ -360,6 +370,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     if (!aligned(q, 16)) return MOE_ERR_INVALID_ARG;
   if (dims->d_s > 0 && !aligned(W_shared, 16)) return MOE_ERR_INVALID_ARG;
   if (dims->router_bias != nullptr && !aligned(dims->router_bias, 16)) return MOE_ERR_INVALID_ARG;
+  if (dims->selection_bias != nullptr && !aligned(dims->selection_bias, 16))
+    return MOE_ERR_INVALID_ARG;
 
   const Plan P = make_plan(dims, E, k, cf);
   if (dims->workspace == nullptr || !aligned(dims->workspace, 256) ||

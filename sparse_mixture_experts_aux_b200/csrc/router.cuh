@@ -347,11 +347,14 @@ __host__ __device__ constexpr size_t route_smem_bytes(int E) {
   return (size_t)ROUTE_WARPS * E * 8 + (size_t)2 * ROUTE_RANK_GROUPS * E * 4;
 }
 
+enum { GATE_RENORM = 0, GATE_RAW = 1, GATE_SIGMOID = 2 };
+
 template <int NV>
-__global__ void __launch_bounds__(256) route_kernel(
-    float* __restrict__ logits, int splits, const float* __restrict__ bias, int T, int E, int k,
-    int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int32_t* __restrict__ lrank_out,
-    int32_t* __restrict__ hist, double* __restrict__ psum_part) {
+__global__ void __launch_bounds__(256, 1) route_kernel(
+    float* __restrict__ logits, int splits, const float* __restrict__ bias,
+    const float* __restrict__ sel_bias, int gate_mode, int n_group, int topk_group, int T, int E,
+    int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+    int32_t* __restrict__ lrank_out, int32_t* __restrict__ hist, double* __restrict__ psum_part) {
   extern __shared__ __align__(16) uint8_t route_smem_raw[];
   double* red = reinterpret_cast<double*>(route_smem_raw);  // [ROUTE_WARPS][E]
   uint32_t* bm = reinterpret_cast<uint32_t*>(red + (size_t)ROUTE_WARPS * E);  // [groups][E]
@@ -361,13 +364,16 @@ __global__ void __launch_bounds__(256) route_kernel(
   for (int i = threadIdx.x; i < ROUTE_RANK_GROUPS * E; i += blockDim.x) bm[i] = 0u;
 
   const int t_warp0 = blk * ROUTE_CHUNK + warp * ROUTE_TOK_PER_WARP;
+  const bool grouped = n_group > 1 && topk_group < n_group;
+  const int gsize = grouped ? E / n_group : E;
   double ps[NV];
-  float bv[NV];
+  float bv[NV], sb[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     ps[i] = 0.0;
     const int e = lane + 32 * i;
     bv[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+    sb[i] = (sel_bias != nullptr && e < E) ? sel_bias[e] : 0.f;
   }
 
   // The next token's logits are loaded (and their K-split partials summed, in
@@ -411,21 +417,74 @@ __global__ void __launch_bounds__(256) route_kernel(
         removed |= 1u << i;
       }
     }
-    m = warp_max(m);
-    float ex[NV];
-    float s = 0.f;
+    // probabilities of the balance statistic; affinities in sigmoid mode
+    float prob[NV], aff[NV];
+    if (gate_mode == GATE_SIGMOID) {
+      float ssum = 0.f;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      ex[i] = (lane + 32 * i < E) ? expf(v[i] - m) : 0.f;
-      s += ex[i];
+      for (int i = 0; i < NV; ++i) {
+        aff[i] = (lane + 32 * i < E) ? 1.f / (1.f + expf(-v[i])) : 0.f;
+        ssum += aff[i];
+      }
+      ssum = warp_sum(ssum);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) prob[i] = aff[i] / ssum;
+    } else {
+      m = warp_max(m);
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        prob[i] = (lane + 32 * i < E) ? expf(v[i] - m) : 0.f;
+        aff[i] = 0.f;
+        s += prob[i];
+      }
+      s = warp_sum(s);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) prob[i] = prob[i] / s;
     }
-    s = warp_sum(s);
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-      if (lane + 32 * i < E) ps[i] += (double)(ex[i] / s);
+      if (lane + 32 * i < E) ps[i] += (double)prob[i];
+
+    // selection scores: logit or affinity, plus the selection-only bias
+    float sel[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) sel[i] = (gate_mode == GATE_SIGMOID ? aff[i] : v[i]) + sb[i];
+    if (grouped) {
+      // group g's best score ends up in lane g; the topk_group best lanes win
+      float my_gb = -INFINITY;
+      for (int g = 0; g < n_group; ++g) {
+        float lm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const int e = lane + 32 * i;
+          if (e < E && e / gsize == g) lm = fmaxf(lm, sel[i]);
+        }
+        lm = warp_max(lm);
+        if (lane == g) my_gb = lm;
+      }
+      bool chosen = false;
+      for (int rnd = 0; rnd < topk_group; ++rnd) {
+        float bvv = (lane < n_group && !chosen) ? my_gb : -INFINITY;
+        int bg = (lane < n_group && !chosen) ? lane : 0x7fffffff;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bvv, o);
+          const int og = __shfl_xor_sync(0xffffffffu, bg, o);
+          if (ov > bvv || (ov == bvv && og < bg)) { bvv = ov; bg = og; }
+        }
+        if (lane == bg) chosen = true;
+      }
+      const uint32_t gmask = __ballot_sync(0xffffffffu, chosen);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((gmask >> (e / gsize)) & 1u)) removed |= 1u << i;
+      }
+    }
 
     int my_e = 0;
-    float my_v = 0.f;
+    float my_g = 0.f;  // the chosen expert's gate input: logit, probability or affinity
     for (int sl = 0; sl < k; ++sl) {
       float best_v = -INFINITY;
       int best_e = 0x7fffffff;
@@ -433,7 +492,7 @@ __global__ void __launch_bounds__(256) route_kernel(
       for (int i = 0; i < NV; ++i) {
         if (!((removed >> i) & 1u)) {
           const int e = lane + 32 * i;
-          if (v[i] > best_v || (v[i] == best_v && e < best_e)) { best_v = v[i]; best_e = e; }
+          if (sel[i] > best_v || (sel[i] == best_v && e < best_e)) { best_v = sel[i]; best_e = e; }
         }
       }
 #pragma unroll
@@ -442,15 +501,28 @@ __global__ void __launch_bounds__(256) route_kernel(
         const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
         if (ov > best_v || (ov == best_v && oe < best_e)) { best_v = ov; best_e = oe; }
       }
-      if (lane == sl) { my_e = best_e; my_v = best_v; }
-      if ((best_e & 31) == lane) removed |= 1u << (best_e >> 5);
+      const int bi = best_e >> 5;
+      float gin = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (i == bi) gin = gate_mode == GATE_RENORM ? v[i] : (gate_mode == GATE_RAW ? prob[i] : aff[i]);
+      gin = __shfl_sync(0xffffffffu, gin, best_e & 31);
+      if (lane == sl) { my_e = best_e; my_g = gin; }
+      if ((best_e & 31) == lane) removed |= 1u << bi;
     }
-    const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-    const float z = (lane < k) ? expf(my_v - v0) : 0.f;
-    const float zs = warp_sum(z);
+    float gate;
+    if (gate_mode == GATE_RENORM) {
+      const float vmax = warp_max(lane < k ? my_g : -INFINITY);
+      const float z = (lane < k) ? expf(my_g - vmax) : 0.f;
+      gate = z / warp_sum(z);
+    } else if (gate_mode == GATE_RAW) {
+      gate = my_g;
+    } else {
+      gate = my_g / warp_sum(lane < k ? my_g : 0.f);
+    }
     if (lane < k) {
       idx_out[(size_t)t * k + lane] = my_e;
-      gate_out[(size_t)t * k + lane] = z / zs;
+      gate_out[(size_t)t * k + lane] = gate;
     }
   }
 #pragma unroll

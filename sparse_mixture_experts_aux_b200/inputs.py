@@ -13,6 +13,8 @@ Recipe (the same for every workload):
   * W_d    ~ N(0, 1/d_e)       [E, d, d_e]
   * shared ~ same, width d_s, packed [gate (d_s x d) | up (d_s x d) | down (d x d_s)]
   * skewed router bias b_e = -1.2 * ln(e + 1) for the Zipf-skewed workload
+  * selection-only bias (routing variants) ~ U(-0.05, 0.05) per expert, fp32, from
+    its own seed: a stand-in for a learned balancing bias
 "N(0, 1/fan_in)" is read as variance 1/fan_in.
 """
 from __future__ import annotations
@@ -38,6 +40,10 @@ class Workload:
     capacity_factor: float = 0.0  # <= 0: no capacity limit
     zipf_bias: bool = False      # add b_e = -1.2 ln(e+1) to the router logits
     seed: int = 0
+    gate_mode: int = 0           # 0 renormalised softmax, 1 raw softmax, 2 sigmoid
+    selection_bias: bool = False  # draw a selection-only per-expert bias
+    n_group: int = 0             # group-limited selection (0/1 = none)
+    topk_group: int = 0
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -96,7 +102,13 @@ def make_inputs(w: Workload, device: str = "cpu", x_seed_offset: int = 0) -> dic
         W_shared = torch.cat([sg.reshape(-1), su.reshape(-1), sd.reshape(-1)]).to(dt)
     x = make_x(w, device, x_seed_offset)
     bias = zipf_router_bias(E).to(device) if w.zipf_bias else None
-    return dict(x=x, W_r=W_r, W_g=W_g, W_u=W_u, W_d=W_d, W_shared=W_shared, router_bias=bias)
+    sel = None
+    if w.selection_bias:
+        gs = torch.Generator(device="cpu")
+        gs.manual_seed(20_000 + w.seed)
+        sel = (torch.rand(E, generator=gs, dtype=torch.float32) * 0.1 - 0.05).to(device)
+    return dict(x=x, W_r=W_r, W_g=W_g, W_u=W_u, W_d=W_d, W_shared=W_shared, router_bias=bias,
+                selection_bias=sel)
 
 
 def make_x(w: Workload, device: str = "cpu", seed_offset: int = 0, T: Optional[int] = None) -> torch.Tensor:

@@ -31,12 +31,17 @@ class Workspace:
 
 
 def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, stream, events,
-              wait_timeout_ns: int = 0):
+              wait_timeout_ns: int = 0, routing: Optional[dict] = None):
     T, d = x.shape
     d_e = W_g.shape[1]
+    routing = routing or {}
     return _lib.make_dims(T, d, d_e, d_s, dtype_code(x.dtype), router_bias, ws,
                           ws.numel() if ws is not None else 0, stream, events,
-                          wait_timeout_ns=wait_timeout_ns)
+                          wait_timeout_ns=wait_timeout_ns,
+                          gate_mode=routing.get("gate_mode", 0),
+                          selection_bias=routing.get("selection_bias"),
+                          n_group=routing.get("n_group", 0),
+                          topk_group=routing.get("topk_group", 0))
 
 
 def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Tensor,
@@ -44,12 +49,15 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
             capacity_factor: float = 0.0, router_bias: Optional[torch.Tensor] = None,
             d_s: int = 0, workspace: Optional[Workspace] = None, stream=None, events=None,
             y: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
-            counts: Optional[torch.Tensor] = None, wait_timeout_ns: int = 0):
+            counts: Optional[torch.Tensor] = None, wait_timeout_ns: int = 0,
+            gate_mode: int = 0, selection_bias: Optional[torch.Tensor] = None,
+            n_group: int = 0, topk_group: int = 0):
     """Run the routed MoE FFN layer; returns (y, aux[1] fp32, counts[E] int32) on x's device.
 
     Shapes: x [T, d]; W_r [E, d] fp32; W_g, W_u [E, d_e, d]; W_d [E, d, d_e];
     W_shared packed [gate d_s*d | up d_s*d | down d*d_s] when d_s > 0.
     wait_timeout_ns: limit of the GEMM kernels' device-side waits (0 = library default).
+    gate_mode / selection_bias / n_group / topk_group: routing variants (include/moe.h).
     """
     for name, t in (("x", x), ("W_r", W_r), ("W_g", W_g), ("W_u", W_u), ("W_d", W_d)):
         if not t.is_cuda:
@@ -63,12 +71,14 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
     elif isinstance(stream, torch.cuda.Stream):
         stream = stream.cuda_stream
     workspace = workspace or Workspace()
-    probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events)
+    routing = dict(gate_mode=gate_mode, selection_bias=selection_bias, n_group=n_group,
+                   topk_group=topk_group)
+    probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events, routing=routing)
     nbytes = _lib.moe_workspace_size(probe, E, k, capacity_factor)
     if nbytes == 0:
         raise _lib.MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
     ws = workspace.get(nbytes, dev)
-    dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns)
+    dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns, routing)
     y = torch.empty_like(x) if y is None else y
     aux = torch.empty(1, dtype=torch.float32, device=dev) if aux is None else aux
     counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts

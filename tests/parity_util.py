@@ -19,7 +19,9 @@ def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None):
     ws = ws or Workspace()
     y, aux, counts = forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"],
                              inp["W_shared"], k=w.k, capacity_factor=w.capacity_factor,
-                             router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws)
+                             router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws,
+                             gate_mode=w.gate_mode, selection_bias=inp.get("selection_bias"),
+                             n_group=w.n_group, topk_group=w.topk_group)
     torch.cuda.synchronize()
     assert moe_get_device_status() == 0, "a device-side wait timed out"
     views = routing_views(ws.buf, inp["x"], inp["W_g"], w.E, w.k, w.capacity_factor, w.d_s)
@@ -36,8 +38,11 @@ def run_oracle(w: Workload, inp: dict, rows=None) -> O.OracleResult:
     shared = None
     if w.d_s:
         shared = tuple(t.cpu() for t in split_shared(inp["W_shared"], w.d, w.d_s))
+    sel = inp.get("selection_bias")
     return O.moe_forward(x, inp["W_r"].cpu(), expert, w.k, layer_capacity_factor(w), bias, shared,
-                         rows)
+                         rows, gate_mode=w.gate_mode,
+                         selection_bias=sel.cpu() if sel is not None else None,
+                         n_group=max(w.n_group, 1), topk_group=max(w.topk_group, 1))
 
 
 def layer_capacity_factor(w: Workload) -> float:

@@ -98,7 +98,12 @@ def test_workspace_size_and_layout(lib):
     (8, 2, dict(T=-1), _lib.MOE_ERR_INVALID_ARG),
     (8, 2, dict(d=0), _lib.MOE_ERR_INVALID_ARG),
     (8, 2, dict(dtype=7), _lib.MOE_ERR_INVALID_ARG),
-    (8, 2, dict(gate_mode=1), _lib.MOE_ERR_UNSUPPORTED),
+    (8, 2, dict(gate_mode=7), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(n_group=3, topk_group=1), _lib.MOE_ERR_INVALID_ARG),   # 3 does not divide E
+    (8, 2, dict(n_group=4, topk_group=5), _lib.MOE_ERR_INVALID_ARG),   # more groups than exist
+    (8, 4, dict(n_group=4, topk_group=1), _lib.MOE_ERR_INVALID_ARG),   # k > experts in 1 group
+    (64, 2, dict(n_group=64, topk_group=2), _lib.MOE_ERR_UNSUPPORTED),  # n_group above 32
+    (8, 2, dict(n_group=-1), _lib.MOE_ERR_INVALID_ARG),
 ])
 def test_forward_rejects_bad_shapes_on_host(lib, E, k, kw, want):
     d = _dims(**kw)
@@ -135,6 +140,18 @@ def test_forward_rejects_bad_pointers_on_host(lib):
     assert call(dims=skew) == _lib.MOE_ERR_WORKSPACE
     assert _lib.moe_forward(None, good, good, good, good, good, None, 8, 2, 0.0, good, good, good,
                             check=False) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_routing_variants_are_accepted_on_host(lib):
+    for kw in (dict(gate_mode=1), dict(gate_mode=2), dict(gate_mode=2, n_group=4, topk_group=2),
+               dict(n_group=8, topk_group=8)):
+        d = _dims(**kw)
+        assert _lib.moe_workspace_size(d, 8, 2, 0.0) > 0, kw
+        st = _lib.moe_forward(d, 16, 16, 16, 16, 16, None, 8, 2, 0.0, 16, 16, 16, check=False)
+        assert st == _lib.MOE_ERR_WORKSPACE, kw  # valid; only the workspace is missing
+    assert _lib.moe_forward(_dims(selection_bias=(1 << 20) + 4), 1 << 20, 1 << 20, 1 << 20,
+                            1 << 20, 1 << 20, None, 8, 2, 0.0, 1 << 20, 1 << 20, 1 << 20,
+                            check=False) == _lib.MOE_ERR_INVALID_ARG  # misaligned bias
 
 
 def test_binding_refuses_cpu_tensors():
