@@ -134,6 +134,27 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+template <int EPI, int AR>
+bool tc_attr() {
+  return cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<EPI, AR>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moe::tc::TcShape<AR>::SMEM_BYTES) == cudaSuccess;
+}
+
+// 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32).
+template <int EPI>
+void launch_tc(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
+               const moe::tc::TcParams& tp) {
+  using namespace moe::tc;
+  if (ar == 32)
+    tc_grouped_gemm_kernel<EPI, 32><<<grid, NUM_THREADS, TcShape<32>::SMEM_BYTES, st>>>(maps, tp);
+  else if (ar == 64)
+    tc_grouped_gemm_kernel<EPI, 64><<<grid, NUM_THREADS, TcShape<64>::SMEM_BYTES, st>>>(maps, tp);
+  else
+    tc_grouped_gemm_kernel<EPI, 128><<<grid, NUM_THREADS, TcShape<128>::SMEM_BYTES, st>>>(maps,
+                                                                                           tp);
+}
+
 template <int EPI>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg{};
@@ -181,11 +202,9 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         return MOE_ERR_CUDA;
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
-    const int smem = moe::tc::SMEM_BYTES;
-    if (cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!tc_attr<moe::tc::EPI_SWIGLU_TC, 128>() || !tc_attr<moe::tc::EPI_SCALE_TC, 128>() ||
+        !tc_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64>() ||
+        !tc_attr<moe::tc::EPI_SWIGLU_TC, 32>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32>())
       return MOE_ERR_CUDA;
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
         !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
@@ -419,19 +438,23 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     const bool pair_up = rows_per_expert >= 2048;
     const bool pair_down = rows_per_expert >= 512;
 #endif
+    // activation box of the 1-CTA kernel: no expert (and no dense group) holds more
+    // than T rows, so small batches load only that many
+    const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
     int32_t* pair_start = reinterpret_cast<int32_t*>(ws + P.o_pair_start);
     constexpr int HB = 128;  // rows of B each CTA of a pair loads
     constexpr int BNp = moe::tc2::BN;
     cudaLaunchAttribute attr[1];
     {
       const int brows = pair_up ? HB : moe::tc::BN / 2;
+      const int abox = pair_up ? moe::tc::BM : arows;
       moe::tc::TcMaps up;
       memset(&up, 0, sizeof(up));
-      bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, moe::tc::BM, 2) &&
+      bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, abox, 2) &&
                 encode_map(&up.b0[0], W_g, P.d, P.de, E, brows, 3) &&
                 encode_map(&up.b1[0], W_u, P.d, P.de, E, brows, 3);
       if (P.ds)
-        ok = ok && encode_map(&up.a[1], x, P.d, P.T, 1, moe::tc::BM, 2) &&
+        ok = ok && encode_map(&up.a[1], x, P.d, P.T, 1, abox, 2) &&
              encode_map(&up.b0[1], sg, P.d, P.ds, 1, brows, 3) &&
              encode_map(&up.b1[1], sg + sh_n, P.d, P.ds, 1, brows, 3);
       if (!ok) return MOE_ERR_CUDA;
@@ -460,20 +483,20 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         if (P.ds)
           tp.g[1] = {nullptr, 1, T, (P.ds + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
                      P.d / moe::tc::BK, P.ds, hs, nullptr};
-        moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>
-            <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(up, tp);
+        launch_tc<moe::tc::EPI_SWIGLU_TC>(arows, num_sms, st, up, tp);
       }
       tm.at(9);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     }
     {
       const int brows = pair_down ? HB : moe::tc::BN;
+      const int abox = pair_down ? moe::tc::BM : arows;
       moe::tc::TcMaps dn;
       memset(&dn, 0, sizeof(dn));
-      bool ok = encode_map(&dn.a[0], h, P.de, P.rows_max, 1, moe::tc::BM, 2) &&
+      bool ok = encode_map(&dn.a[0], h, P.de, P.rows_max, 1, abox, 2) &&
                 encode_map(&dn.b0[0], W_d, P.de, P.d, E, brows, 3);
       if (P.ds)
-        ok = ok && encode_map(&dn.a[1], hs, P.ds, P.T, 1, moe::tc::BM, 2) &&
+        ok = ok && encode_map(&dn.a[1], hs, P.ds, P.T, 1, abox, 2) &&
              encode_map(&dn.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, brows, 3);
       if (!ok) return MOE_ERR_CUDA;
       dn.b1[0] = dn.b0[0];
@@ -503,8 +526,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         if (P.ds)
           tp.g[1] = {nullptr, 1, T, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.ds / moe::tc::BK,
                      P.d, ys, nullptr};
-        moe::tc::tc_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>
-            <<<num_sms, moe::tc::NUM_THREADS, moe::tc::SMEM_BYTES, st>>>(dn, tp);
+        launch_tc<moe::tc::EPI_SCALE_TC>(arows, num_sms, st, dn, tp);
       }
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;

@@ -33,17 +33,33 @@ constexpr int BM = 128;            // rows per tile (= ROW_TILE)
 constexpr int BN = 256;            // accumulator columns per tile (UMMA N)
 constexpr int BK = 64;             // K per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;         // K of one tcgen05.mma kind::f16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_E + 1);
 
 static_assert(BM == ROW_TILE, "GEMM row tile must match the segment padding");
+
+// Shape of the 1-CTA kernel for an activation box of AR rows. AR = 128 is the
+// general case. When every expert holds at most 32 (64) rows, which holds for
+// any batch of at most that many tokens, the box shrinks to AR rows, so a
+// stage is smaller and the ring deeper: more weight bytes in flight for the
+// weight-streaming (decode) shapes. The M = 128 MMA still reads 128 rows from
+// the A slot. The rows past AR are stale bytes inside the same stage buffer;
+// their results land only in the padding rows of the expert's 128-row segment,
+// and the epilogue warps that own them skip their stores.
+template <int AR>
+struct TcShape {
+  static_assert(AR == 128 || AR == 64 || AR == 32, "activation box rows");
+  static constexpr int A_BYTES = AR * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = AR == 128 ? 4 : (AR == 64 ? 5 : 6);
+  static constexpr int SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_E + 1);
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+  static_assert(A_BYTES % 1024 == 0, "B slot must stay 1024-byte aligned");
+};
 
 enum { EPI_SWIGLU_TC = 0, EPI_SCALE_TC = 1 };
 
@@ -272,9 +288,12 @@ __device__ __forceinline__ TileInfo decode_tile(long long tile, long long tiles0
   return ti;
 }
 
-template <int EPI>
+template <int EPI, int AR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  constexpr int STAGES = TcShape<AR>::STAGES;
+  constexpr int A_BYTES = TcShape<AR>::A_BYTES;
+  constexpr int STAGE_BYTES = TcShape<AR>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -415,6 +434,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = ti.row0 + r_in_tile;
       const bool row_ok = (g.tile_start != nullptr) || row < g.rows;
       const uint32_t tb = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
+      if (quad * 32 < AR) {
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.N;
       if (EPI == EPI_SWIGLU_TC) {
 #pragma unroll 1
@@ -453,6 +473,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      }  // quad * 32 < AR
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));

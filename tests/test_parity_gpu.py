@@ -26,6 +26,9 @@ SMALL = [
     Workload("bf16 single expert", 130, 128, 1, 128, 1, seed=18),
     Workload("bf16 E=1024 k=32", 64, 64, 1024, 64, 32, seed=19),
     Workload("bf16 one token", 1, 256, 8, 256, 2, seed=20),
+    # batches of <= 64 / <= 32 tokens use the short activation boxes
+    Workload("bf16 T=48 shared expert, 64-row box", 48, 256, 8, 256, 2, d_s=128, seed=33),
+    Workload("bf16 T=20 capacity, 32-row box", 20, 192, 4, 192, 2, capacity_factor=1.5, seed=34),
     Workload("bf16 shared+capacity", 700, 256, 8, 256, 2, d_s=256, capacity_factor=0.8, seed=21),
     Workload("fp32 shared+capacity", 333, 128, 8, 96, 2, "f32", d_s=64, capacity_factor=0.7, seed=22),
     Workload("fp32 ragged", 257, 96, 5, 160, 3, "f32", seed=23),
