@@ -52,6 +52,8 @@ __all__ = [
     "topk_margin", "capacity_limit", "capacity_keep", "silu", "swiglu_ffn",
     "GATE_RENORM", "GATE_RAW", "GATE_SIGMOID", "sigmoid_affinity", "balance_probs",
     "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
+    "E4M3_MAX", "e4m3_round", "e4m3_encode", "e4m3_decode", "quantize_rows_fp8",
+    "dequantize_rows_fp8",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
     "moe_param_count", "active_flops", "OracleResult",
 ]
@@ -364,6 +366,72 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
                         capacity=C, keep=keep, probsum=probsum, aux=aux,
                         margin=margin, rows=rows, y=y[rows],
                         dropped_fraction=dropped_fraction(counts, C, T, k))
+
+
+# ----------------------------------------------------------------------------
+# FP8 expert weights (weight-only quantisation)
+#   AI Engineering Illustrated "Mixture of Experts", "Trade-offs to weigh" (at
+#   small batch MoE inference is limited by reading weights; quantising the
+#   expert weights, as gpt-oss does with MXFP4, attacks that directly) and
+#   jacopoparretti "Mixture of experts, token by token", "Memory" (DeepSeek-V3
+#   ships its weights in FP8, one byte per parameter).
+# Readings (the pages fix no format details): R11 the 8-bit format is E4M3
+#   (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, largest
+#   finite value 448, no infinities), rounded to nearest-even and saturated to
+#   +-448; R12 one fp32 scale per output row, scale = fp32(absmax / 448) (1 for
+#   an all-zero row), code = E4M3(fp32(w / scale)); the layer uses
+#   code_value * scale.
+# ----------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Nearest E4M3 value (ties to even), saturated to +-448, as float64.
+    The spacing is 2^-9 below 2^-6 (subnormals) and 2^(e-3) in [2^e, 2^(e+1))."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    q = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (e - 3))
+    r = np.minimum(np.rint(a / q) * q, E4M3_MAX)
+    return np.copysign(r, v)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """uint8 codes (sign << 7 | exponent << 3 | mantissa) of E4M3 values."""
+    r = e4m3_round(v)
+    a = np.abs(r)
+    sign = np.signbit(r).astype(np.uint8) << 7
+    normal = a >= 2.0 ** -6
+    e = np.floor(np.log2(np.where(normal, a, 1.0))).astype(np.int64)
+    mant_n = np.rint(a / 2.0 ** e * 8 - 8).astype(np.int64)
+    mant_s = np.rint(a / 2.0 ** -9).astype(np.int64)
+    code = np.where(normal, ((e + 7) << 3) | mant_n, mant_s)
+    return (sign | code.astype(np.uint8)).astype(np.uint8)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of E4M3 codes (0x7F / 0xFF, the NaN codes, never occur)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return s * val
+
+
+def quantize_rows_fp8(w):
+    """Per-row E4M3 quantisation (R12) of a [rows, cols] matrix; returns
+    (codes uint8 [rows, cols], scales fp32 [rows])."""
+    w32 = np.asarray(_f64(w), dtype=np.float32)
+    absmax = np.abs(w32).max(axis=1)
+    scales = np.where(absmax > 0, absmax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    ratio = (w32 / scales[:, None]).astype(np.float32)
+    return e4m3_encode(ratio), scales
+
+
+def dequantize_rows_fp8(codes, scales) -> np.ndarray:
+    """The weights the layer computes with: code value times the row scale (fp64, exact)."""
+    return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
 
 
 # ----------------------------------------------------------------------------
