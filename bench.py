@@ -41,7 +41,10 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral",
                     choices=["mixtral", "deepseek_v3", "switch_zipf", "decode", "tiny_fp32",
-                             "mixtral_profile"])
+                             "mixtral_profile", "decode_profile"])
+    ap.add_argument("--weights", choices=["dtype", "fp8"], default="dtype",
+                    help="expert weights in the activation dtype, or E4M3 codes with per-row "
+                         "scales (quantised once by the library before timing)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -51,7 +54,7 @@ def workload_by_name(name):
     from sparse_mixture_experts_aux_b200 import inputs as I
     return {"mixtral": I.MIXTRAL, "deepseek_v3": I.DEEPSEEK_V3, "switch_zipf": I.SWITCH_ZIPF,
             "decode": I.MIXTRAL_DECODE, "tiny_fp32": I.TINY_F32,
-            "mixtral_profile": I.MIXTRAL_PROFILE}[name]
+            "mixtral_profile": I.MIXTRAL_PROFILE, "decode_profile": I.DECODE_PROFILE}[name]
 
 
 def load_peaks():
@@ -209,7 +212,8 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from sparse_mixture_experts_aux_b200 import (KERNEL_NAMES, MOE_NUM_KERNELS, Workspace,
-                                                 forward, _lib, moe_get_device_status)
+                                                 forward, _lib, moe_get_device_status,
+                                                 quantize_fp8)
     from sparse_mixture_experts_aux_b200.events import KernelEvents
     from sparse_mixture_experts_aux_b200.inputs import make_inputs, make_x
     from oracle import moe_oracle as O  # cpu_baseline leg only
@@ -225,12 +229,21 @@ def run_ours(args, rank, world, local_rank):
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     counts = torch.empty(w.E, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    fp8 = args.weights == "fp8"
+    scales = None
+    if fp8:  # one-off weight preparation, untimed
+        parts = []
+        for name in ("W_g", "W_u", "W_d"):
+            inp[name], sc = quantize_fp8(inp[name])
+            parts.append(sc.reshape(-1))
+        scales = torch.cat(parts)
+        torch.cuda.synchronize()
 
     def call(i, events=None):
         forward(xs[i % R], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["W_shared"],
                 k=w.k, capacity_factor=w.capacity_factor, router_bias=inp["router_bias"],
                 d_s=w.d_s, workspace=ws, stream=stream, events=events, y=y, aux=aux,
-                counts=counts)
+                counts=counts, weight_scales=scales)
 
     def barrier():
         if world > 1:
@@ -275,10 +288,12 @@ def run_ours(args, rank, world, local_rank):
     kept = int(cnt.sum() if C is None else sum(min(int(c), C) for c in cnt))
     touched = int(sum(1 for c in cnt if (c if C is None else min(int(c), C)) > 0))
     esz = 2 if w.dtype == "bf16" else 4
+    wsz = 1 if fp8 else esz  # bytes per expert weight (+ 4 per row of scales with FP8)
     flops_up = 2 * kept * w.d * 2 * w.d_e + (2 * w.T * w.d * 2 * w.d_s if w.d_s else 0)
     flops_down = 2 * kept * w.d_e * w.d + (2 * w.T * w.d_s * w.d if w.d_s else 0)
     flops_active = flops_up + flops_down
-    w_bytes = touched * 3 * w.d * w.d_e * esz + 3 * w.d * w.d_s * esz + w.E * w.d * 4
+    w_bytes = (touched * 3 * w.d * w.d_e * wsz + (touched * 2 * (w.d_e + w.d) * 4 if fp8 else 0)
+               + 3 * w.d * w.d_s * esz + w.E * w.d * 4)
     act_bytes = 2 * w.T * w.d * esz
     peaks, peaks_src = load_peaks()
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -289,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
     k_up = per_kernel[4]
     # the gate/up kernel's own roofline: its FLOPs at tensor peak vs its
     # algorithmic bytes (touched gate+up weights, permuted rows in, H out) at HBM
-    bytes_up = (touched * 2 * w.d * w.d_e * esz + (2 * w.d * w.d_s * esz if w.d_s else 0)
+    bytes_up = (touched * 2 * w.d * w.d_e * wsz + (touched * 2 * w.d_e * 4 if fp8 else 0)
+                + (2 * w.d * w.d_s * esz if w.d_s else 0)
                 + (kept + (w.T if w.d_s else 0)) * (w.d + w.d_e) * esz)
     up_bound = "tensor" if flops_up / (tensor_peak * 1e12) >= bytes_up / (hbm_peak * 1e9) else "hbm"
     if up_bound == "tensor":
@@ -304,8 +320,9 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": config_of(w, "inputs larger than L2: %.2f GB of expert weights streamed per "
-                               "step; x rotates over %d batches" % (w_bytes / 1e9, R)),
+        "config": dict(config_of(w, "inputs larger than L2: %.2f GB of expert weights streamed "
+                                    "per step; x rotates over %d batches" % (w_bytes / 1e9, R)),
+                       weights="e4m3 codes + fp32 row scales" if fp8 else w.dtype),
         "roofline": {"bound": up_bound, "kernel": KERNEL_NAMES[4], "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": None,
                      "algorithmic_per_launch": work, "peak_source": peak_note},
@@ -332,7 +349,9 @@ def run_ours(args, rank, world, local_rank):
         nbytes = ws.buf.numel()
         dims = _lib.make_dims(w.T, w.d, w.d_e, w.d_s,
                               _lib.MOE_BF16 if w.dtype == "bf16" else _lib.MOE_F32,
-                              inp["router_bias"], ws.buf, nbytes, stream.cuda_stream)
+                              inp["router_bias"], ws.buf, nbytes, stream.cuda_stream,
+                              weight_format=_lib.MOE_WEIGHTS_FP8 if fp8 else _lib.MOE_WEIGHTS_DTYPE,
+                              weight_scales=scales)
 
         def e2e_call(i):
             _lib.moe_forward_host_io(dims, x_host[i % 2], x_dev, inp["W_r"], inp["W_g"],

@@ -103,6 +103,20 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 #define MOE_GATE_RAW 1
 #define MOE_GATE_SIGMOID 2
 
+/*
+ * FP8 expert weights (weight-only quantisation). At small batch, an MoE layer
+ * is limited by reading expert weights, and quantising them attacks that
+ * directly (AI Engineering Illustrated "Mixture of Experts", "Trade-offs to
+ * weigh"; jacopoparretti "Mixture of experts, token by token", "Memory":
+ * DeepSeek-V3 ships FP8 weights). Format: E4M3 (bias 7, largest finite 448,
+ * round-to-nearest-even, saturating); one fp32 scale per output row,
+ * scale = absmax(row) / 448 (1 for an all-zero row), code = E4M3(w / scale).
+ * The layer computes with code * scale: the GEMMs stream the codes and
+ * dequantise them to bf16 on chip, so activations keep bf16 precision.
+ */
+#define MOE_WEIGHTS_DTYPE 0
+#define MOE_WEIGHTS_FP8 1
+
 typedef struct {
   int64_t T;                 /* tokens in this call (0 allowed: empty batch) */
   int32_t d;                 /* model width */
@@ -125,6 +139,12 @@ typedef struct {
   int32_t n_group;           /* group-limited selection: experts form n_group contiguous
                                 groups of E / n_group; 0 or 1 = no groups */
   int32_t topk_group;        /* groups a token may pick from (1 <= topk_group <= n_group) */
+  int32_t weight_format;     /* MOE_WEIGHTS_DTYPE (0): W_g, W_u, W_d in `dtype`;
+                                MOE_WEIGHTS_FP8 (1): E4M3 codes (uint8) with per-row scales,
+                                see moe_quantize_fp8 (bf16 activations, no shared expert) */
+  const float* weight_scales; /* MOE_WEIGHTS_FP8: device fp32, the per-row scales of the three
+                                 stacks one after another: W_g [E*d_e], W_u [E*d_e],
+                                 W_d [E*d] (what moe_quantize_fp8 writes for each stack) */
   uint64_t wait_timeout_ns;  /* limit of each device-side mbarrier wait in the GEMM
                                 kernels; 0 = default (4 s). A tiny value makes the waits
                                 expire on purpose: the kernels then record
@@ -145,8 +165,9 @@ MOE_API int64_t moe_capacity(int64_t T, int E, int k, float capacity_factor);
  * Forward pass of the routed MoE FFN layer (see top of file).
  *   x        device [T, d]            dtype
  *   W_r      device [E, d]            fp32 (the router's d x E matrix, stored expert-major)
- *   W_g, W_u device [E, d_e, d]       dtype (nn.Linear weight layout: K contiguous)
- *   W_d      device [E, d, d_e]       dtype
+ *   W_g, W_u device [E, d_e, d]       dtype (nn.Linear weight layout: K contiguous),
+ *                                    or uint8 E4M3 codes with MOE_WEIGHTS_FP8
+ *   W_d      device [E, d, d_e]       dtype (or uint8 codes)
  *   W_shared device, packed [gate (d_s x d) | up (d_s x d) | down (d x d_s)], or
  *            NULL when dims->d_s == 0
  *   y        device [T, d]            dtype, written (every row)
@@ -207,6 +228,32 @@ MOE_API moe_status moe_get_device_status(void);
 
 /* Static, human-readable name of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
+
+/*
+ * Quantise `rows` rows of `cols` weights (device, `dtype` = MOE_BF16 or MOE_F32,
+ * row-major) to E4M3 codes (device uint8 [rows, cols]) and per-row scales
+ * (device fp32 [rows]) with the rule above, asynchronously on `stream`. For a
+ * routed expert stack, W_g [E, d_e, d] is rows = E * d_e, cols = d (likewise
+ * W_u), and W_d [E, d, d_e] is rows = E * d, cols = d_e. Writing the three
+ * stacks' scales one after another gives moe_dims.weight_scales. Returns
+ * MOE_ERR_INVALID_ARG for null pointers, cols not a multiple of 16, rows < 0
+ * or a bad dtype (nothing is launched), MOE_ERR_CUDA on launch failure.
+ */
+MOE_API moe_status moe_quantize_fp8(const void* w, int32_t dtype, int64_t rows, int32_t cols,
+                                    uint8_t* codes, float* scales, void* stream);
+
+/*
+ * The weights an FP8 layer computes with: out[r][c] = value(codes[r][c]) *
+ * scales[r] (device fp32 [rows, cols]), each code decoded exactly by the
+ * routine the GEMM kernels use, the product rounded once to fp32. For
+ * checking a quantised stack or materialising it. Codes 0x7F / 0xFF (E4M3
+ * NaN, never written by moe_quantize_fp8) are outside the contract. Returns
+ * MOE_ERR_INVALID_ARG for null pointers, rows < 0, cols not a multiple of 16,
+ * or codes / out not 16-byte aligned (nothing is launched), MOE_ERR_CUDA on
+ * launch failure.
+ */
+MOE_API moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales, int64_t rows,
+                                      int32_t cols, float* out, void* stream);
 
 /*
  * moe_forward for callers that cannot allocate device memory. The pages have

@@ -22,12 +22,13 @@ MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_GATE_RENORM, MOE_GATE_RAW, MOE_GATE_SIGMOID = 0, 1, 2
+MOE_WEIGHTS_DTYPE, MOE_WEIGHTS_FP8 = 0, 1
 MOE_NUM_KERNELS = 7
 KERNEL_NAMES = ("router_logits", "route", "scan", "scatter", "gate_up_swiglu", "down_scale", "combine")
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_forward", "moe_forward_host_io",
             "moe_workspace_layout", "moe_get_device_status", "moe_status_string",
-            "moe_forward_no_alloc")
+            "moe_forward_no_alloc", "moe_quantize_fp8", "moe_dequantize_fp8")
 
 
 class moe_dims(ctypes.Structure):
@@ -46,6 +47,8 @@ class moe_dims(ctypes.Structure):
         ("selection_bias", ctypes.c_void_p),
         ("n_group", ctypes.c_int32),
         ("topk_group", ctypes.c_int32),
+        ("weight_format", ctypes.c_int32),
+        ("weight_scales", ctypes.c_void_p),
         ("wait_timeout_ns", ctypes.c_uint64),
     ]
 
@@ -104,6 +107,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_get_device_status.restype = i32
     lib.moe_status_string.argtypes = [i32]
     lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_quantize_fp8.argtypes = [vp, i32, ctypes.c_int64, i32, vp, vp, vp]
+    lib.moe_quantize_fp8.restype = i32
+    lib.moe_dequantize_fp8.argtypes = [vp, vp, ctypes.c_int64, i32, vp, vp]
+    lib.moe_dequantize_fp8.restype = i32
     _lib = lib
     return lib
 
@@ -127,7 +134,8 @@ def _ptr(t) -> int:
 def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, router_bias=None,
               workspace=None, workspace_bytes: int = 0, stream: int = 0, events=None,
               gate_mode: int = 0, wait_timeout_ns: int = 0, selection_bias=None,
-              n_group: int = 0, topk_group: int = 0) -> moe_dims:
+              n_group: int = 0, topk_group: int = 0, weight_format: int = MOE_WEIGHTS_DTYPE,
+              weight_scales=None) -> moe_dims:
     """Fill a moe_dims. `events` is a ctypes array of cudaEvent_t handles or None."""
     dims = moe_dims()
     dims.T, dims.d, dims.d_e, dims.d_s = int(T), int(d), int(d_e), int(d_s)
@@ -140,6 +148,8 @@ def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, rou
     dims.wait_timeout_ns = int(wait_timeout_ns)
     dims.selection_bias = _ptr(selection_bias) or None
     dims.n_group, dims.topk_group = int(n_group), int(topk_group)
+    dims.weight_format = int(weight_format)
+    dims.weight_scales = _ptr(weight_scales) or None
     return dims
 
 
@@ -194,3 +204,15 @@ def moe_forward_no_alloc(dims: moe_dims, x, W_r, W_g, W_u, W_d, W_shared, E: int
 
 def moe_get_device_status() -> int:
     return int(load().moe_get_device_status())
+
+
+def moe_quantize_fp8(w, dtype: int, rows: int, cols: int, codes, scales, stream: int = 0) -> int:
+    """Raw call: returns the status code."""
+    return int(load().moe_quantize_fp8(_ptr(w) or None, int(dtype), int(rows), int(cols),
+                                       _ptr(codes) or None, _ptr(scales) or None, int(stream) or None))
+
+
+def moe_dequantize_fp8(codes, scales, rows: int, cols: int, out, stream: int = 0) -> int:
+    """Raw call: returns the status code."""
+    return int(load().moe_dequantize_fp8(_ptr(codes) or None, _ptr(scales) or None, int(rows),
+                                         int(cols), _ptr(out) or None, int(stream) or None))

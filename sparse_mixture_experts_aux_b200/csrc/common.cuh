@@ -81,6 +81,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Cycle budget for a wait limited to `ns` nanoseconds, counted on the SM's own
+// cycle counter (a cheap register read, unlike %globaltimer, whose read sits on
+// the critical path of every wait that does not succeed at once). 2 cycles per
+// ns is above the SM's top clock, so the limit in wall time is never shorter
+// than asked; at lower clocks it is longer.
+__device__ __forceinline__ uint64_t wait_cycles(unsigned long long ns) {
+  return ns > (1ull << 61) ? (1ull << 62) : 2ull * ns;
+}
+
 __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + __expf(-a)); }
 
 }  // namespace moe

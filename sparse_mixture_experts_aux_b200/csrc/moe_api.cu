@@ -13,6 +13,7 @@
 #include "permute.cuh"
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
+#include "tc_f8_gemm.cuh"
 
 namespace {
 
@@ -65,6 +66,10 @@ moe_status check_dims(const moe_dims* dims, int E, int k, float cf) {
   }
   if (dims->T * static_cast<int64_t>(k) >= (int64_t(1) << 31) ||
       dims->T * static_cast<int64_t>(E) >= (int64_t(1) << 40))
+    return MOE_ERR_UNSUPPORTED;
+  if (dims->weight_format != MOE_WEIGHTS_DTYPE && dims->weight_format != MOE_WEIGHTS_FP8)
+    return MOE_ERR_INVALID_ARG;
+  if (dims->weight_format == MOE_WEIGHTS_FP8 && (dims->dtype != MOE_BF16 || dims->d_s != 0))
     return MOE_ERR_UNSUPPORTED;
   const int mult = dims->dtype == MOE_BF16 ? 64 : 32;
   if (dims->d % mult || dims->d_e % mult || dims->d_s % mult) return MOE_ERR_UNSUPPORTED;
@@ -141,6 +146,26 @@ bool tc_attr() {
                               moe::tc::TcShape<AR>::SMEM_BYTES) == cudaSuccess;
 }
 
+template <int EPI, int AR>
+bool f8_attr() {
+  return cudaFuncSetAttribute(moe::tcf8::tc_f8_grouped_gemm_kernel<EPI, AR>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moe::tcf8::F8Shape<AR>::SMEM_BYTES) == cudaSuccess;
+}
+
+template <int EPI>
+void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
+               const moe::tcf8::F8Params& fp) {
+  using namespace moe::tcf8;
+  if (ar == 32)
+    tc_f8_grouped_gemm_kernel<EPI, 32><<<grid, NUM_THREADS, F8Shape<32>::SMEM_BYTES, st>>>(maps, fp);
+  else if (ar == 64)
+    tc_f8_grouped_gemm_kernel<EPI, 64><<<grid, NUM_THREADS, F8Shape<64>::SMEM_BYTES, st>>>(maps, fp);
+  else
+    tc_f8_grouped_gemm_kernel<EPI, 128>
+        <<<grid, NUM_THREADS, F8Shape<128>::SMEM_BYTES, st>>>(maps, fp);
+}
+
 // 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32).
 template <int EPI>
 void launch_tc(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
@@ -206,6 +231,10 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64>() ||
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 32>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32>())
       return MOE_ERR_CUDA;
+    if (!f8_attr<moe::tc::EPI_SWIGLU_TC, 128>() || !f8_attr<moe::tc::EPI_SCALE_TC, 128>() ||
+        !f8_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !f8_attr<moe::tc::EPI_SCALE_TC, 64>() ||
+        !f8_attr<moe::tc::EPI_SWIGLU_TC, 32>() || !f8_attr<moe::tc::EPI_SCALE_TC, 32>())
+      return MOE_ERR_CUDA;
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
         !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
       return MOE_ERR_CUDA;
@@ -259,6 +288,24 @@ bool encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, 
   const CUresult r =
       g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// FP8 code tensor map over [outer][mid][inner] codes (inner a multiple of 16),
+// box {128 codes, box_rows, 1} (full 128-byte lines), 128-byte swizzle. The
+// codes are described to the TMA unit as 32-bit words (4 codes each): the
+// bytes land exactly where a uint8 map would put them, in a quarter of the
+// elements.
+bool encode_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                   uint32_t box_rows) {
+  cuuint64_t dims[3] = {inner / 4, mid, outer};
+  cuuint64_t strides[2] = {inner, inner * mid};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::tcf8::F8Shape<128>::QK / 4), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -391,6 +438,9 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   if (dims->router_bias != nullptr && !aligned(dims->router_bias, 16)) return MOE_ERR_INVALID_ARG;
   if (dims->selection_bias != nullptr && !aligned(dims->selection_bias, 16))
     return MOE_ERR_INVALID_ARG;
+  if (dims->weight_format == MOE_WEIGHTS_FP8 &&
+      (dims->weight_scales == nullptr || !aligned(dims->weight_scales, 4)))
+    return MOE_ERR_INVALID_ARG;
 
   const Plan P = make_plan(dims, E, k, cf);
   if (dims->workspace == nullptr || !aligned(dims->workspace, 256) ||
@@ -424,6 +474,46 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     const size_t sh_n = static_cast<size_t>(P.ds) * P.d;
     const int ng = P.ds ? 2 : 1;
 
+    if (dims->weight_format == MOE_WEIGHTS_FP8) {
+      // FP8 expert weights: 1-CTA kernels that dequantise the weight tiles on chip
+      const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
+      const float* sc = dims->weight_scales;
+      const size_t gsz = static_cast<size_t>(E) * P.de;
+      moe::tc::TcMaps up, dn;
+      memset(&up, 0, sizeof(up));
+      memset(&dn, 0, sizeof(dn));
+      const bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, arows, 2) &&
+                      encode_map_u8(&up.b0[0], W_g, P.d, P.de, E, moe::tc::BN / 2) &&
+                      encode_map_u8(&up.b1[0], W_u, P.d, P.de, E, moe::tc::BN / 2) &&
+                      encode_map(&dn.a[0], h, P.de, P.rows_max, 1, arows, 2) &&
+                      encode_map_u8(&dn.b0[0], W_d, P.de, P.d, E, moe::tc::BN);
+      if (!ok) return MOE_ERR_CUDA;
+      dn.b1[0] = dn.b0[0];
+      moe::tcf8::F8Params fu{};
+      fu.timeout_ns = wait_tmo;
+      fu.drain_timeout_ns = kDrainTimeoutNs;
+      fu.grp.g = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                  P.d / moe::tc::BK, P.de, h, nullptr};
+      fu.grp.scale0 = sc;
+      fu.grp.scale1 = sc + gsz;
+      fu.grp.scale_stride = P.de;
+      moe::tcf8::F8Params fd{};
+      fd.timeout_ns = wait_tmo;
+      fd.drain_timeout_ns = kDrainTimeoutNs;
+      fd.grp.g = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
+                  P.d, yrows, rowgate};
+      fd.grp.scale0 = sc + 2 * gsz;
+      fd.grp.scale1 = sc + 2 * gsz;
+      fd.grp.scale_stride = P.d;
+      tm.at(8);
+      launch_f8<moe::tc::EPI_SWIGLU_TC>(arows, num_sms, st, up, fu);
+      tm.at(9);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+      tm.at(10);
+      launch_f8<moe::tc::EPI_SCALE_TC>(arows, num_sms, st, dn, fd);
+      tm.at(11);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    } else {
     // (4) gate/up projection + SwiGLU, (5) down projection scaled by the gates.
     // CTA-pair tiles (256 rows) cut the operand traffic per SM by a third but
     // pair up the 128-row tiles of each expert, so an expert with an odd tile
@@ -531,6 +621,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     }
+    }  // bf16 weights
     // (6) combine
     tm.at(12);
     {
@@ -682,6 +773,37 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_SCRATCH_LIMIT: return "MOE_ERR_SCRATCH_LIMIT";
   }
   return "MOE_STATUS_UNKNOWN";
+}
+
+moe_status moe_quantize_fp8(const void* w, int32_t dtype, int64_t rows, int32_t cols,
+                            uint8_t* codes, float* scales, void* stream) {
+  if (w == nullptr || codes == nullptr || scales == nullptr || rows < 0 || cols < 1 ||
+      cols % 16 != 0 || (dtype != MOE_BF16 && dtype != MOE_F32) || !aligned(scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(rows < 8192 ? rows : 8192);
+  if (dtype == MOE_BF16)
+    moe::tcf8::quantize_rows_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), rows, cols, codes, scales);
+  else
+    moe::tcf8::quantize_rows_fp8_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float*>(w), rows, cols, codes, scales);
+  return launched();
+}
+
+moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales, int64_t rows,
+                              int32_t cols, float* out, void* stream) {
+  if (codes == nullptr || scales == nullptr || out == nullptr || rows < 0 || cols < 1 ||
+      cols % 16 != 0 || !aligned(codes, 16) || !aligned(out, 16) || !aligned(scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  const int64_t n = rows * (cols / 16);
+  const int64_t blocks = (n + 255) / 256;
+  moe::tcf8::dequantize_rows_fp8_kernel<<<static_cast<unsigned>(blocks < 16384 ? blocks : 16384),
+                                          256, 0, static_cast<cudaStream_t>(stream)>>>(
+      codes, scales, rows, cols, out);
+  return launched();
 }
 
 moe_status moe_forward_no_alloc(const moe_dims* dims, const void* x, const float* W_r,

@@ -150,12 +150,13 @@ __device__ __noinline__ bool wait_pair(uint32_t bar, uint32_t parity, volatile i
                                        uint32_t peer_abort_cluster,
                                        unsigned long long timeout_ns) {
   if (tc::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_cycles(timeout_ns);
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (tc::mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 1u) {
+    if ((it & 15u) == 1u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
+      if (static_cast<uint64_t>(clock64() - t0) > limit) {
         atomicOr(&g_dev_error, DEVERR_TIMEOUT);
         *abort_flag = 1;
         st_cluster_u32(peer_abort_cluster, 1u);

@@ -121,13 +121,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_cycles(timeout_ns);
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     // try_wait itself suspends for a while, so check on the first re-poll too
-    if ((it & 127u) == 1u) {
+    if ((it & 15u) == 1u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
+      if (static_cast<uint64_t>(clock64() - t0) > limit) {
         atomicOr(&g_dev_error, DEVERR_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -141,10 +142,11 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
 __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity,
                                         unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_cycles(timeout_ns);
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 1u && globaltimer_ns() - t0 > timeout_ns) {
+    if ((it & 15u) == 1u && static_cast<uint64_t>(clock64() - t0) > limit) {
       atomicOr(&g_dev_error, DEVERR_TIMEOUT);
       return false;
     }

@@ -16,6 +16,12 @@ Recipe (the same for every workload):
   * selection-only bias (routing variants) ~ U(-0.05, 0.05) per expert, fp32, from
     its own seed: a stand-in for a learned balancing bias
 "N(0, 1/fan_in)" is read as variance 1/fan_in.
+
+FP8 expert weights drawn directly as data (make_fp8_weights): E4M3 codes
+uniform over the 254 finite codes (a random sign, a magnitude field uniform in
+0..0x7E), and one fp32 scale per output row ~ U(0.5, 1.5) / (100 sqrt(fan_in)),
+so that the weights' RMS is near 1/sqrt(fan_in) (the RMS of a uniform finite
+code is about 104).
 """
 from __future__ import annotations
 
@@ -68,6 +74,9 @@ ALL_WORKLOADS = (TINY_F32, MIXTRAL, DEEPSEEK_V3, SWITCH_ZIPF, MIXTRAL_DECODE)
 # hardware-counter captures of the same kernels.
 MIXTRAL_PROFILE = Workload("mixtral-shape-profile T=2048 d=4096 E=2 d_e=14336 k=2",
                            2048, 4096, 2, 14336, 2, seed=1)
+# The decode shape with 2 experts (about 0.7 GB of bf16 weights), likewise.
+DECODE_PROFILE = Workload("decode-shape-profile T=32 d=4096 E=2 d_e=14336 k=2",
+                          32, 4096, 2, 14336, 2, seed=4)
 
 
 def zipf_router_bias(E: int) -> torch.Tensor:
@@ -123,3 +132,24 @@ def split_shared(W_shared: torch.Tensor, d: int, d_s: int):
     """View the packed shared-expert buffer as (gate [d_s,d], up [d_s,d], down [d,d_s])."""
     n = d_s * d
     return (W_shared[:n].view(d_s, d), W_shared[n:2 * n].view(d_s, d), W_shared[2 * n:3 * n].view(d, d_s))
+
+
+def make_fp8_weights(w: Workload, device: str = "cpu") -> dict:
+    """Random E4M3 expert weights for workload `w`: uint8 codes W_g, W_u [E, d_e, d],
+    W_d [E, d, d_e] and weight_scales fp32 [E*d_e | E*d_e | E*d] (that order)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(30_000 + w.seed)
+    E, d, de = w.E, w.d, w.d_e
+
+    def codes(shape):
+        mag = torch.randint(0, 0x7F, shape, generator=gen, device=device, dtype=torch.int32)
+        sign = torch.randint(0, 2, shape, generator=gen, device=device, dtype=torch.int32) << 7
+        return (mag | sign).to(torch.uint8)
+
+    def scales(n, fan_in):
+        u = torch.rand(n, generator=gen, device=device, dtype=torch.float32) + 0.5
+        return u / (100.0 * math.sqrt(fan_in))
+
+    W_g, W_u, W_d = codes((E, de, d)), codes((E, de, d)), codes((E, d, de))
+    sc = torch.cat([scales(E * de, d), scales(E * de, d), scales(E * d, de)])
+    return dict(W_g=W_g, W_u=W_u, W_d=W_d, weight_scales=sc)

@@ -31,17 +31,20 @@ class Workspace:
 
 
 def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, stream, events,
-              wait_timeout_ns: int = 0, routing: Optional[dict] = None):
+              wait_timeout_ns: int = 0, routing: Optional[dict] = None, weight_scales=None):
     T, d = x.shape
     d_e = W_g.shape[1]
     routing = routing or {}
+    fp8 = W_g.dtype == torch.uint8
     return _lib.make_dims(T, d, d_e, d_s, dtype_code(x.dtype), router_bias, ws,
                           ws.numel() if ws is not None else 0, stream, events,
                           wait_timeout_ns=wait_timeout_ns,
                           gate_mode=routing.get("gate_mode", 0),
                           selection_bias=routing.get("selection_bias"),
                           n_group=routing.get("n_group", 0),
-                          topk_group=routing.get("topk_group", 0))
+                          topk_group=routing.get("topk_group", 0),
+                          weight_format=_lib.MOE_WEIGHTS_FP8 if fp8 else _lib.MOE_WEIGHTS_DTYPE,
+                          weight_scales=weight_scales)
 
 
 def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Tensor,
@@ -51,11 +54,13 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
             y: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
             counts: Optional[torch.Tensor] = None, wait_timeout_ns: int = 0,
             gate_mode: int = 0, selection_bias: Optional[torch.Tensor] = None,
-            n_group: int = 0, topk_group: int = 0):
+            n_group: int = 0, topk_group: int = 0, weight_scales: Optional[torch.Tensor] = None):
     """Run the routed MoE FFN layer; returns (y, aux[1] fp32, counts[E] int32) on x's device.
 
     Shapes: x [T, d]; W_r [E, d] fp32; W_g, W_u [E, d_e, d]; W_d [E, d, d_e];
     W_shared packed [gate d_s*d | up d_s*d | down d*d_s] when d_s > 0.
+    FP8 expert weights: W_g, W_u, W_d as uint8 E4M3 codes (quantize_fp8) and
+    weight_scales = their per-row scales concatenated [W_g | W_u | W_d] (bf16 x).
     wait_timeout_ns: limit of the GEMM kernels' device-side waits (0 = library default).
     gate_mode / selection_bias / n_group / topk_group: routing variants (include/moe.h).
     """
@@ -73,17 +78,50 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
     workspace = workspace or Workspace()
     routing = dict(gate_mode=gate_mode, selection_bias=selection_bias, n_group=n_group,
                    topk_group=topk_group)
-    probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events, routing=routing)
+    if W_g.dtype == torch.uint8:
+        if weight_scales is None or not weight_scales.is_cuda or weight_scales.dtype != torch.float32:
+            raise RuntimeError("FP8 weights need weight_scales: a CUDA fp32 tensor")
+    probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events, routing=routing,
+                      weight_scales=weight_scales)
     nbytes = _lib.moe_workspace_size(probe, E, k, capacity_factor)
     if nbytes == 0:
         raise _lib.MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
     ws = workspace.get(nbytes, dev)
-    dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns, routing)
+    dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns, routing,
+                     weight_scales)
     y = torch.empty_like(x) if y is None else y
     aux = torch.empty(1, dtype=torch.float32, device=dev) if aux is None else aux
     counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
     _lib.moe_forward(dims, x, W_r, W_g, W_u, W_d, W_shared, E, k, capacity_factor, y, aux, counts)
     return y, aux, counts
+
+
+def quantize_fp8(w: torch.Tensor, stream=None):
+    """E4M3 codes (uint8, w's shape) and per-row fp32 scales of a CUDA weight
+    tensor whose last dimension is the row (include/moe.h, moe_quantize_fp8)."""
+    if not w.is_cuda or not w.is_contiguous():
+        raise RuntimeError("w must be a contiguous CUDA tensor")
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    st = torch.cuda.current_stream(w.device).cuda_stream if stream is None else stream
+    rc = _lib.moe_quantize_fp8(w, dtype_code(w.dtype), rows, cols, codes, scales, st)
+    if rc != _lib.MOE_OK:
+        raise _lib.MoeError(rc, "moe_quantize_fp8")
+    return codes, scales
+
+
+def dequantize_fp8(codes: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """fp32 weights code * scale, as the FP8 layer computes with them (moe_dequantize_fp8)."""
+    cols = codes.shape[-1]
+    rows = codes.numel() // cols
+    out = torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    st = torch.cuda.current_stream(codes.device).cuda_stream if stream is None else stream
+    rc = _lib.moe_dequantize_fp8(codes, scales, rows, cols, out, st)
+    if rc != _lib.MOE_OK:
+        raise _lib.MoeError(rc, "moe_dequantize_fp8")
+    return out
 
 
 def routing_views(ws: torch.Tensor, x: torch.Tensor, W_g: torch.Tensor, E: int, k: int,

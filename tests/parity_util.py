@@ -15,25 +15,38 @@ GATE_TOL = 1e-6      # absolute, on gates
 Y_TOL = {"f32": 1e-4, "bf16": 2e-2}  # max|err| <= tol * max(1, |ref|)
 
 
-def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None):
+def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None, fp8: dict | None = None):
+    """fp8: E4M3 codes W_g, W_u, W_d and weight_scales (device) to use instead of
+    the dtype weights in `inp`."""
     ws = ws or Workspace()
-    y, aux, counts = forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"],
+    src = fp8 if fp8 is not None else inp
+    y, aux, counts = forward(inp["x"], inp["W_r"], src["W_g"], src["W_u"], src["W_d"],
                              inp["W_shared"], k=w.k, capacity_factor=w.capacity_factor,
                              router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws,
                              gate_mode=w.gate_mode, selection_bias=inp.get("selection_bias"),
-                             n_group=w.n_group, topk_group=w.topk_group)
+                             n_group=w.n_group, topk_group=w.topk_group,
+                             weight_scales=fp8["weight_scales"] if fp8 is not None else None)
     torch.cuda.synchronize()
     assert moe_get_device_status() == 0, "a device-side wait timed out"
     views = routing_views(ws.buf, inp["x"], inp["W_g"], w.E, w.k, w.capacity_factor, w.d_s)
     return y, aux, counts, views
 
 
-def run_oracle(w: Workload, inp: dict, rows=None) -> O.OracleResult:
+def run_oracle(w: Workload, inp: dict, rows=None, fp8: dict | None = None) -> O.OracleResult:
+    """fp8: as in run_gpu; the oracle then computes with code * scale (its own
+    dequantisation, fp64)."""
     x = inp["x"].cpu()
     bias = inp["router_bias"].cpu() if inp["router_bias"] is not None else None
 
     def expert(e):
-        return inp["W_g"][e].cpu(), inp["W_u"][e].cpu(), inp["W_d"][e].cpu()
+        if fp8 is None:
+            return inp["W_g"][e].cpu(), inp["W_u"][e].cpu(), inp["W_d"][e].cpu()
+        E, de, d = w.E, w.d_e, w.d
+        sc = fp8["weight_scales"]
+        parts = ((fp8["W_g"][e], sc[e * de:(e + 1) * de]),
+                 (fp8["W_u"][e], sc[E * de + e * de:E * de + (e + 1) * de]),
+                 (fp8["W_d"][e], sc[2 * E * de + e * d:2 * E * de + (e + 1) * d]))
+        return tuple(O.dequantize_rows_fp8(c.cpu().numpy(), s.cpu().numpy()) for c, s in parts)
 
     shared = None
     if w.d_s:
@@ -139,3 +152,17 @@ def check_workload(w: Workload, sample: int | None = None, seed: int = 0) -> dic
         rows = np.sort(rng.choice(w.T, size=sample, replace=False))
     ref = run_oracle(w, inp, rows)
     return compare(w, gpu, ref)
+
+
+def oracle_quantized_weights(inp: dict, device="cuda") -> dict:
+    """E4M3 codes and scales of the drawn dtype weights, computed by the oracle's
+    quantiser on the CPU, in the layer's FP8 input layout."""
+    out, scales = {}, []
+    for name in ("W_g", "W_u", "W_d"):
+        wt = inp[name].float().cpu().numpy()
+        n, r, c = wt.shape
+        codes, sc = O.quantize_rows_fp8(wt.reshape(-1, c))
+        out[name] = torch.from_numpy(codes.reshape(n, r, c)).to(device)
+        scales.append(torch.from_numpy(sc))
+    out["weight_scales"] = torch.cat(scales).to(device)
+    return out

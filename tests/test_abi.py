@@ -104,6 +104,9 @@ def test_workspace_size_and_layout(lib):
     (8, 4, dict(n_group=4, topk_group=1), _lib.MOE_ERR_INVALID_ARG),   # k > experts in 1 group
     (64, 2, dict(n_group=64, topk_group=2), _lib.MOE_ERR_UNSUPPORTED),  # n_group above 32
     (8, 2, dict(n_group=-1), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(weight_format=5), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(weight_format=1, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),  # FP8: bf16 x
+    (8, 2, dict(weight_format=1, d_s=128), _lib.MOE_ERR_UNSUPPORTED),  # FP8: no shared expert
 ])
 def test_forward_rejects_bad_shapes_on_host(lib, E, k, kw, want):
     d = _dims(**kw)
@@ -152,6 +155,24 @@ def test_routing_variants_are_accepted_on_host(lib):
     assert _lib.moe_forward(_dims(selection_bias=(1 << 20) + 4), 1 << 20, 1 << 20, 1 << 20,
                             1 << 20, 1 << 20, None, 8, 2, 0.0, 1 << 20, 1 << 20, 1 << 20,
                             check=False) == _lib.MOE_ERR_INVALID_ARG  # misaligned bias
+
+
+def test_fp8_weights_validated_on_host(lib):
+    g = 1 << 20
+    fwd = lambda d: _lib.moe_forward(d, g, g, g, g, g, None, 8, 2, 0.0, g, g, g, check=False)
+    assert fwd(_dims(weight_format=1)) == _lib.MOE_ERR_INVALID_ARG          # scales missing
+    assert fwd(_dims(weight_format=1, weight_scales=g + 2)) == _lib.MOE_ERR_INVALID_ARG
+    assert _lib.moe_workspace_size(_dims(weight_format=1, weight_scales=g), 8, 2, 0.0) > 0
+    assert fwd(_dims(weight_format=1, weight_scales=g)) == _lib.MOE_ERR_WORKSPACE  # valid
+    # quantiser and dequantiser: argument checks on the host, nothing launched
+    for args in [(0, 1, 4, 64, g, g), (g, 1, 4, 64, 0, g), (g, 1, 4, 64, g, 0), (g, 1, 4, 24, g, g),
+                 (g, 1, -1, 64, g, g), (g, 9, 4, 64, g, g), (g, 1, 4, 0, g, g)]:
+        assert _lib.moe_quantize_fp8(*args) == _lib.MOE_ERR_INVALID_ARG, args
+    assert _lib.moe_quantize_fp8(g, 1, 0, 64, g, g) == _lib.MOE_OK  # no rows: nothing to do
+    for args in [(0, g, 4, 64, g), (g, 0, 4, 64, g), (g, g, 4, 64, 0), (g, g, 4, 40, g),
+                 (g + 8, g, 4, 64, g), (g, g, 4, 64, g + 4), (g, g, -2, 64, g)]:
+        assert _lib.moe_dequantize_fp8(*args) == _lib.MOE_ERR_INVALID_ARG, args
+    assert _lib.moe_dequantize_fp8(g, g, 0, 64, g) == _lib.MOE_OK
 
 
 def test_binding_refuses_cpu_tensors():

@@ -8,7 +8,7 @@ import torch
 
 from sparse_mixture_experts_aux_b200 import Workspace, _lib, forward, moe_get_device_status
 from sparse_mixture_experts_aux_b200.inputs import Workload, make_inputs
-from tests.parity_util import compare, run_gpu, run_oracle
+from tests.parity_util import compare, oracle_quantized_weights, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -36,3 +36,21 @@ def test_expired_waits_are_reported_and_the_context_survives(w):
         assert moe_get_device_status() == _lib.MOE_OK  # reading it resets it
     gpu = run_gpu(w, inp, ws)  # default limit: completes and matches the oracle
     compare(w, gpu, run_oracle(w, inp))
+
+
+@pytest.mark.parametrize("w", [
+    Workload("timeout fp8 32-row box", 20, 256, 4, 320, 2, seed=44),
+    Workload("timeout fp8 128-row box", 700, 256, 4, 320, 2, seed=45),
+], ids=lambda w: w.name)
+def test_expired_waits_fp8_kernels(w):
+    inp = make_inputs(w, device="cuda")
+    fp8 = oracle_quantized_weights(inp)
+    ws = Workspace()
+    for _ in range(3):
+        forward(inp["x"], inp["W_r"], fp8["W_g"], fp8["W_u"], fp8["W_d"], None, k=w.k,
+                workspace=ws, weight_scales=fp8["weight_scales"], wait_timeout_ns=1)
+        torch.cuda.synchronize()
+        assert moe_get_device_status() == _lib.MOE_ERR_DEVICE_TIMEOUT
+        assert moe_get_device_status() == _lib.MOE_OK
+    gpu = run_gpu(w, inp, ws, fp8=fp8)
+    compare(w, gpu, run_oracle(w, inp, fp8=fp8))
