@@ -111,8 +111,11 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * DeepSeek-V3 ships FP8 weights). Format: E4M3 (bias 7, largest finite 448,
  * round-to-nearest-even, saturating); one fp32 scale per output row,
  * scale = absmax(row) / 448 (1 for an all-zero row), code = E4M3(w / scale).
- * The layer computes with code * scale: the GEMMs stream the codes and
- * dequantise them to bf16 on chip, so activations keep bf16 precision.
+ * The layer computes with code * scale: the GEMMs stream the codes and decode
+ * them on chip to fp16 (exact), and run fp16 x fp16 -> fp32 on the tensor
+ * cores, so the routed activations and H are held in fp16 on this path
+ * (exact for bf16 inputs with 2^-14 <= |x| <= 65504; larger magnitudes
+ * saturate at 65504). x and y stay bf16.
  */
 #define MOE_WEIGHTS_DTYPE 0
 #define MOE_WEIGHTS_FP8 1

@@ -407,8 +407,13 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   {
     const int nvec = static_cast<int>(static_cast<size_t>(P.d) * sizeof(TX) / 16);
     dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
-    moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
-                                                  base, tile_start, slot, rowgate, xp);
+    if (dims->weight_format == MOE_WEIGHTS_FP8)  // the FP8-weight GEMMs read fp16 rows
+      moe::scatter_kernel<TX, true><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate,
+                                                          lrank, base, tile_start, slot, rowgate,
+                                                          xp);
+    else
+      moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
+                                                    base, tile_start, slot, rowgate, xp);
   }
   tm.at(7);
   return launched();

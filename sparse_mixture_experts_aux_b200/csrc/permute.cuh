@@ -10,6 +10,7 @@
 // capacity limit".
 #pragma once
 #include "common.cuh"
+#include <cuda_fp16.h>
 
 namespace moe {
 
@@ -25,7 +26,25 @@ constexpr int PERMUTE_CHUNK_VECS = 32 * PERMUTE_VPL;
 // tile_start[e]*ROW_TILE + rank (blocks with blockIdx.y == 0 record it). The
 // chunk of the token's row is then copied to every kept position with 16-byte
 // loads and stores (coalesced across the warp).
-template <typename TX>
+// bf16 x 8 -> fp16 x 8, saturating at +-65504 (the FP8-weight GEMMs run
+// f16 x f16; every bf16 value in [2^-14, 65504] converts exactly).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& u) {
+  float f[8];
+  Vec16<__nv_bfloat16>::unpack(u, f);
+  uint4 r;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = fminf(fmaxf(f[2 * i], -65504.f), 65504.f);
+    const float b = fminf(fmaxf(f[2 * i + 1], -65504.f), 65504.f);
+    const __half2 h = __floats2half2_rn(a, b);
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return r;
+}
+
+// TO_F16: write the rows as fp16 (bf16 input only), for the FP8-weight GEMMs.
+template <typename TX, bool TO_F16 = false>
 __global__ void __launch_bounds__(256) scatter_kernel(
     const TX* __restrict__ x, int d, int T, int k, int E, int64_t C,
     const int32_t* __restrict__ idx, const float* __restrict__ gate,
@@ -54,7 +73,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int p = __shfl_sync(0xffffffffu, mypos, s);
     if (p < 0) continue;
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)p * d);
-    for (int c = c_begin + lane; c < c_end; c += 32) st_v4(dst + c, ld_nc_v4(src + c));
+    for (int c = c_begin + lane; c < c_end; c += 32) {
+      const uint4 v = ld_nc_v4(src + c);
+      st_v4(dst + c, TO_F16 ? bf16x8_to_f16x8(v) : v);
+    }
   }
 }
 

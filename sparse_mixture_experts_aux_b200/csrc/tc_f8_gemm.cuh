@@ -2,28 +2,35 @@
 //
 // The weights stay in HBM as E4M3 codes with one fp32 scale per output row,
 // so a weight-streaming (decode) pass reads half the bytes of bf16 weights.
-// The activations stay bf16, and the tensor cores run kind::f16 exactly as in
-// the bf16 kernel. Three shared-memory rings:
-//   A  bf16 activation boxes (AR rows x 64), one per 64-deep K step; TMA in,
-//      released by the MMA's commit
-//   Q  FP8 weight tiles, 256 rows x 128 codes (two K steps, full 128-byte
-//      lines, 128-byte swizzle); TMA in, released by the converter warps as
-//      soon as they have turned both halves into bf16, so the weight stream
-//      never waits for the tensor cores
-//   B  bf16 weight tiles (256 x 64, the 128-byte-swizzled K-major layout the
-//      MMA reads); written by 8 converter warps, released by the MMA's commit
-// The MMA (one thread) reads A and B, accumulates fp32 in TMEM; the epilogue
-// multiplies by the per-row weight scale, then applies SwiGLU or the gate
-// scale as the bf16 kernel does.
+// The MMAs run kind::f16 with fp16 operands: E4M3 codes convert to fp16 exactly
+// with one instruction per pair, the permuted activations arrive as fp16 (the
+// scatter kernel converts them; exact for 2^-14 <= |x| <= 65504, saturating
+// above), and this kernel stores H as fp16. Three shared-memory rings:
+//   Q  FP8 weight tiles, 256 rows x 128 codes (two 64-deep K chunks, full
+//      128-byte lines, 128-byte swizzle); TMA in, released by the converter
+//      warps once decoded, so the weight stream never waits for the MMAs
+//   A  stages of CH fp16 activation boxes (TMA), released by the MMA commit;
+//      deeper than S, so the boxes (L2 hits) are fetched well ahead
+//   S  stages of CH decoded fp16 weight tiles (256 x 64 each, the
+//      128-byte-swizzled K-major layout the MMA reads, written by 8 converter
+//      warps); released by the MMA commit
+// The MMA thread waits once and commits once per stage. Every barrier
+// operation of one thread is a serial step of roughly a hundred cycles, so
+// per 64-deep chunk it matters how many each role issues: with two chunks per
+// stage the MMA thread spends 1 wait + 8 MMAs + 1 commit per 128-deep step.
+// The epilogue multiplies by the per-row weight scale, then applies SwiGLU or
+// the gate scale as the bf16 kernel does.
 // Sources: AI Engineering Illustrated "Mixture of Experts", "Trade-offs to
 // weigh" (small-batch MoE inference is limited by reading weights; quantising
 // the expert weights attacks that directly); jacopoparretti "Mixture of
 // experts, token by token", "Memory" (DeepSeek-V3 ships FP8 weights).
 //
 // Synchronisation (all waits bounded, as in the bf16 kernel):
-//   afull[a] producer expect_tx + TMA bytes;   aempty[a] 1 MMA commit
-//   qfull[q] producer expect_tx + TMA bytes;   qempty[q] 8 converter-warp arrivals
-//   bfull[b] 8 converter-warp arrivals;        bempty[b] 1 MMA commit
+//   qfull[q]  Q producer expect_tx + TMA bytes;   qempty[q] 8 converter-warp arrivals
+//   afull[a]  A producer expect_tx + TMA bytes (waited by the first converter
+//             warp);                                 aempty[a] 1 MMA commit
+//   full[s]   8 converter-warp arrivals (the first one after afull[a]): activations
+//             landed and weights decoded;          empty[s]  1 MMA commit
 //   tfull/tempty/done as in the bf16 kernel.
 #pragma once
 #include "tc_gemm.cuh"
@@ -39,8 +46,9 @@ using tc::UMMA_K;
 using tc::TcMaps;
 
 constexpr int CONV_WARPS = 8;
-// warp 0 producer, 1 MMA, 2-5 epilogue, 6-13 converters
-constexpr int NUM_THREADS = (6 + CONV_WARPS) * 32;
+// warp 0 activation producer, 1 MMA, 2-5 epilogue, 6-13 converters, 14 weight producer
+constexpr int NUM_THREADS = (7 + CONV_WARPS) * 32;
+constexpr int QPROD_WARP = 6 + CONV_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BAR_BYTES = 256;
 constexpr int CONV_WARP0 = 6;
@@ -48,22 +56,24 @@ constexpr int CONV_WARP0 = 6;
 template <int AR>
 struct F8Shape {
   static_assert(AR == 128 || AR == 64 || AR == 32, "activation box rows");
-  static constexpr int A_BYTES = AR * BK * 2;        // bf16 activation box
+  static constexpr int CH = AR == 128 ? 1 : 2;       // 64-deep K chunks per stage
+  static constexpr int A_SUB = AR * BK * 2;          // fp16 activation box of one chunk
+  static constexpr int B_SUB = BN * BK * 2;          // decoded fp16 weights of one chunk
+  static constexpr int A_BYTES = CH * A_SUB;         // a stage of ring A
+  static constexpr int S_BYTES = CH * B_SUB;         // a stage of ring S (weights)
   static constexpr int QK = 2 * BK;                  // codes per weight row in a Q stage
-  static constexpr int Q_BYTES = BN * QK;            // FP8 weight tile: 256 rows x 128 B
-  static constexpr int B16_BYTES = BN * BK * 2;      // converted bf16 weight tile
-  // a Q stage feeds two K steps, so the activation ring holds two boxes per Q stage
-  static constexpr int NQ = AR == 128 ? 2 : 3;
-  static constexpr int NA = 2 * NQ;
-  static constexpr int NB = AR == 32 ? 3 : 2;
-  static constexpr int RING_BYTES = NA * A_BYTES + NQ * Q_BYTES + NB * B16_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (tc::MAX_E + 1);
+  static constexpr int Q_BYTES = BN * QK;            // 256 rows x 128 B
+  static constexpr int NS = AR == 128 ? 3 : 2;
+  static constexpr int NA = AR == 64 ? 2 : 4;        // activations run ahead of the weights
+  static constexpr int NQ = 2;
+  static constexpr int RING_BYTES = NS * S_BYTES + NA * A_BYTES + NQ * Q_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-  // the M = 128 MMA reads 16 KB from an activation slot; the Q ring follows the
-  // A ring, so the rows beyond AR stay inside this CTA's shared memory
-  static_assert(NA * A_BYTES + NQ * Q_BYTES >= (NA - 1) * A_BYTES + BM * BK * 2,
-                "activation reads stay inside shared memory");
-  static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "1024-byte aligned slots");
+  // the M = 128 MMA reads 16 KB from an A chunk; ring Q follows ring A, so the
+  // rows beyond AR stay inside this CTA's shared memory
+  static_assert(NA * A_BYTES - A_SUB + NQ * Q_BYTES >= BM * BK * 2, "activation reads in bounds");
+  static_assert(A_SUB % 1024 == 0 && S_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0,
+                "1024-byte aligned slots");
 };
 
 struct F8Group {
@@ -79,34 +89,30 @@ struct F8Params {
   unsigned long long drain_timeout_ns;
 };
 
-// Four E4M3 codes (code i in byte i of `w`) -> four bf16 values, as two bf16x2
-// words (codes 0,1 and codes 2,3). Exact for every finite code, with integer
-// operations and one bf16x2 FMA per pair instead of format conversions:
-// the code's sign goes to bf16 bit 15 and its 7 magnitude bits to bits 10..4.
-// Read as bf16, that is the E4M3 value times 2^-120: the 4-bit exponent field
-// sits in the low bits of bf16's 8-bit field (bias 127 instead of 7) and the
-// 3 mantissa bits lead bf16's 7; exponent field 0 (the E4M3 subnormals) lands
-// on bf16 subnormals with the same factor. Multiplying by 2^120 (an FMA with a
-// -0 addend, which keeps the sign of zero) restores the value without rounding.
-// Codes 0x7F / 0xFF (E4M3 NaN) are never written by the quantiser; they would
-// read as +-480.
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
-  return r;
+// Four E4M3 codes (code i in byte i of `w`) -> four fp16 values, as two f16x2
+// words (codes 0,1 and codes 2,3), with the hardware conversion: one
+// instruction per pair, exact for every finite code (E4M3 values, subnormals
+// included, are fp16 values). Per instruction this is a quarter of the work of
+// building bf16 values with integer operations, which is why the FP8-weight
+// GEMMs run f16 x f16: the converters would otherwise bound the kernel.
+// Codes 0x7F / 0xFF (E4M3 NaN) are never written by the quantiser.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
-__device__ __forceinline__ uint32_t bf16x2_scale(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(0x80008000u));
-  return r;
+
+// fp32 pair -> f16x2, saturating at +-65504 (H of the FP8-weight path).
+__device__ __forceinline__ uint32_t f16x2_sat(float a, float b) {
+  const __half2 h = __floats2half2_rn(fminf(fmaxf(a, -65504.f), 65504.f),
+                                      fminf(fmaxf(b, -65504.f), 65504.f));
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  constexpr uint32_t MASK = 0x87F087F0u;       // bf16 sign and bits 10..4, both halves
-  constexpr uint32_t POW2_120 = 0x7B807B80u;   // bf16x2 (2^120, 2^120)
-  // bytes sign-extended to 16-bit halves (prmt selector nibble 8|i: sign of byte i)
-  const uint32_t t01 = prmt(w, 0x9180u), t23 = prmt(w, 0xB3A2u);
-  lo = bf16x2_scale((t01 << 4) & MASK, POW2_120);
-  hi = bf16x2_scale((t23 << 4) & MASK, POW2_120);
+
+// Instruction descriptor, kind::f16 with A and B fp16 (format 0), D fp32.
+__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void fence_async_shared() {
@@ -137,37 +143,42 @@ template <int EPI, int AR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_f8_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const F8Params p) {
   using Sh = F8Shape<AR>;
-  constexpr int NA = Sh::NA, NQ = Sh::NQ, NB = Sh::NB;
+  constexpr int NS = Sh::NS, NA = Sh::NA, NQ = Sh::NQ, CH = Sh::CH;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = tc::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint8_t* a_base = smem;                                   // ring A: NA activation boxes
+  uint8_t* s_base = smem;                                   // ring S: NS decoded weight stages
+  uint8_t* a_base = s_base + NS * Sh::S_BYTES;              // ring A: NA activation stages
   uint8_t* q_base = a_base + NA * Sh::A_BYTES;              // ring Q: NQ x 32 KB FP8 tiles
-  uint8_t* b_base = q_base + NQ * Sh::Q_BYTES;              // ring B: NB x 32 KB bf16 tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::RING_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * (NA + NQ + NB) + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2 * NA + 2 * NQ + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_ts = reinterpret_cast<int32_t*>(smem + Sh::RING_BYTES + BAR_BYTES);
+  // segment starts: read from global memory (L1-cached) by the few threads that
+  // walk tiles, which leaves all of shared memory to the rings
+  const int32_t* s_ts = p.grp.g.tile_start;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t s_0 = tc::smem_addr(s_base);
   const uint32_t a_0 = tc::smem_addr(a_base);
   const uint32_t q_0 = tc::smem_addr(q_base);
-  const uint32_t b_0 = tc::smem_addr(b_base);
   const uint32_t bar0 = tc::smem_addr(bars);
-  auto afull = [&](int i) { return bar0 + 8u * i; };
-  auto aempty = [&](int i) { return bar0 + 8u * (NA + i); };
-  auto qfull = [&](int i) { return bar0 + 8u * (2 * NA + i); };
-  auto qempty = [&](int i) { return bar0 + 8u * (2 * NA + NQ + i); };
-  auto bfull = [&](int i) { return bar0 + 8u * (2 * NA + 2 * NQ + i); };
-  auto bempty = [&](int i) { return bar0 + 8u * (2 * NA + 2 * NQ + NB + i); };
-  constexpr int T0 = 2 * (NA + NQ + NB);
+  auto full = [&](int i) { return bar0 + 8u * i; };
+  auto empty = [&](int i) { return bar0 + 8u * (NS + i); };
+  auto afull = [&](int i) { return bar0 + 8u * (2 * NS + i); };
+  auto aempty = [&](int i) { return bar0 + 8u * (2 * NS + NA + i); };
+  auto qfull = [&](int i) { return bar0 + 8u * (2 * NS + 2 * NA + i); };
+  auto qempty = [&](int i) { return bar0 + 8u * (2 * NS + 2 * NA + NQ + i); };
+  constexpr int T0 = 2 * NS + 2 * NA + 2 * NQ;
   auto tfull = [&](int a) { return bar0 + 8u * (T0 + a); };
   auto tempty = [&](int a) { return bar0 + 8u * (T0 + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (T0 + 4);
 
   const tc::TcGroup& G = p.grp.g;
-  for (int i = threadIdx.x; i <= G.E; i += NUM_THREADS) s_ts[i] = G.tile_start[i];
   if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      tc::mbar_init(full(i), CONV_WARPS);
+      tc::mbar_init(empty(i), 1);
+    }
     for (int i = 0; i < NA; ++i) {
       tc::mbar_init(afull(i), 1);
       tc::mbar_init(aempty(i), 1);
@@ -175,10 +186,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int i = 0; i < NQ; ++i) {
       tc::mbar_init(qfull(i), 1);
       tc::mbar_init(qempty(i), CONV_WARPS);
-    }
-    for (int i = 0; i < NB; ++i) {
-      tc::mbar_init(bfull(i), CONV_WARPS);
-      tc::mbar_init(bempty(i), 1);
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(tfull(a), 1);
@@ -198,82 +205,94 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const long long total = (long long)G.n_tiles * s_ts[G.E];
-  const int kbs = G.k_blocks;
+  const int nck = G.k_blocks;                 // 64-deep K chunks per tile
+  const int nst = (nck + CH - 1) / CH;        // S stages per tile
+  const int nqs = (nck + 1) / 2;              // Q stages per tile
   const unsigned long long tmo = p.timeout_ns, drain_tmo = p.drain_timeout_ns;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    // In issue order: the Q tile of K steps kb and kb + 1, then the two
-    // activation boxes of those steps. A TMA unit serves its copies roughly in
-    // order, so a box issued far behind a deep queue of weight tiles would
-    // arrive late; issued right behind its own tile, it lands with it.
+    // ------------------------------------------------------ activation producer
     if (lane == 0) {
       tc::prefetch_map(&maps.a[0]);
-      tc::prefetch_map(&maps.b0[0]);
-      if (EPI == tc::EPI_SWIGLU_TC) tc::prefetch_map(&maps.b1[0]);
-      int as = 0, qs = 0;
-      uint32_t aph = 0, qph = 0, a_issued = 0, a_par = 0, q_issued = 0, q_par = 0;
+      int as = 0;
+      uint32_t aph = 0, issued = 0, par = 0;
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
-        for (int kb = 0; ok && kb < kbs; ++kb) {
-          if ((kb & 1) == 0) {
-            if (!tc::wait_bounded(qempty(qs), qph ^ 1u, abort_flag, tmo)) { ok = false; break; }
-            const uint32_t dq = q_0 + qs * Sh::Q_BYTES;
-            tc::mbar_expect_tx(qfull(qs), Sh::Q_BYTES);
-            if (EPI == tc::EPI_SWIGLU_TC) {
-              tc::tma_load_3d(dq, &maps.b0[0], qfull(qs), kb * (BK / 4), ti.nb * (BN / 2), ti.e);
-              tc::tma_load_3d(dq + Sh::Q_BYTES / 2, &maps.b1[0], qfull(qs), kb * (BK / 4),
-                              ti.nb * (BN / 2), ti.e);
-            } else {
-              tc::tma_load_3d(dq, &maps.b0[0], qfull(qs), kb * (BK / 4), ti.nb * BN, ti.e);
-            }
-            q_issued |= 1u << qs;
-            q_par = (q_par & ~(1u << qs)) | (qph << qs);
-            if (++qs == NQ) { qs = 0; qph ^= 1u; }
-          }
+        for (int st = 0; st < nst; ++st) {
           if (!tc::wait_bounded(aempty(as), aph ^ 1u, abort_flag, tmo)) { ok = false; break; }
-          tc::mbar_expect_tx(afull(as), Sh::A_BYTES);
-          tc::tma_load_2d(a_0 + as * Sh::A_BYTES, &maps.a[0], afull(as), kb * BK, ti.row0);
-          a_issued |= 1u << as;
-          a_par = (a_par & ~(1u << as)) | (aph << as);
+          const int nv = min(CH, nck - st * CH);
+          tc::mbar_expect_tx(afull(as), nv * Sh::A_SUB);
+          for (int c = 0; c < nv; ++c)
+            tc::tma_load_2d(a_0 + as * Sh::A_BYTES + c * Sh::A_SUB, &maps.a[0], afull(as),
+                            (st * CH + c) * BK, ti.row0);
+          issued |= 1u << as;
+          par = (par & ~(1u << as)) | (aph << as);
           if (++as == NA) { as = 0; aph ^= 1u; }
         }
       }
-      if (!ok) {  // let every copy already issued land before the CTA exits
-        for (int i = 0; i < NQ; ++i)
-          if ((q_issued >> i) & 1u) tc::wait_drain(qfull(i), (q_par >> i) & 1u, drain_tmo);
+      if (!ok)  // let every copy already issued land before the CTA exits
         for (int i = 0; i < NA; ++i)
-          if ((a_issued >> i) & 1u) tc::wait_drain(afull(i), (a_par >> i) & 1u, drain_tmo);
+          if ((issued >> i) & 1u) tc::wait_drain(afull(i), (par >> i) & 1u, drain_tmo);
+    }
+  } else if (warp == QPROD_WARP) {
+    // ---------------------------------------------------------- weight producer
+    if (lane == 0) {
+      tc::prefetch_map(&maps.b0[0]);
+      if (EPI == tc::EPI_SWIGLU_TC) tc::prefetch_map(&maps.b1[0]);
+      int qs = 0;
+      uint32_t qph = 0, issued = 0, par = 0;
+      bool ok = true;
+      for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+        for (int qi = 0; qi < nqs; ++qi) {
+          if (!tc::wait_bounded(qempty(qs), qph ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          const uint32_t dq = q_0 + qs * Sh::Q_BYTES;
+          const int x = qi * (Sh::QK / 4);  // the codes are described as 32-bit words
+          tc::mbar_expect_tx(qfull(qs), Sh::Q_BYTES);
+          if (EPI == tc::EPI_SWIGLU_TC) {
+            tc::tma_load_3d(dq, &maps.b0[0], qfull(qs), x, ti.nb * (BN / 2), ti.e);
+            tc::tma_load_3d(dq + Sh::Q_BYTES / 2, &maps.b1[0], qfull(qs), x, ti.nb * (BN / 2),
+                            ti.e);
+          } else {
+            tc::tma_load_3d(dq, &maps.b0[0], qfull(qs), x, ti.nb * BN, ti.e);
+          }
+          issued |= 1u << qs;
+          par = (par & ~(1u << qs)) | (qph << qs);
+          if (++qs == NQ) { qs = 0; qph ^= 1u; }
+        }
       }
+      if (!ok)
+        for (int i = 0; i < NQ; ++i)
+          if ((issued >> i) & 1u) tc::wait_drain(qfull(i), (par >> i) & 1u, drain_tmo);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = tc::make_idesc(BM, BN);
-      int as = 0, bs = 0;
-      uint32_t aph = 0, bph = 0, acc = 0, acc_phase = 0;
+      constexpr uint32_t IDESC = make_idesc_f16(BM, BN);
+      int ss = 0, as = 0;
+      uint32_t sph = 0, aph = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         if (!tc::wait_bounded(tempty(acc), acc_phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kbs; ++kb) {
-          if (!tc::wait_bounded(afull(as), aph, abort_flag, tmo) ||
-              !tc::wait_bounded(bfull(bs), bph, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
+        for (int st = 0; st < nst; ++st) {
+          if (!tc::wait_bounded(full(ss), sph, abort_flag, tmo)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint64_t ad = tc::sw128_kmajor_desc(a_0 + as * Sh::A_BYTES);
-          const uint64_t bd = tc::sw128_kmajor_desc(b_0 + bs * Sh::B16_BYTES);
+          const int nv = min(CH, nck - st * CH);
+          for (int c = 0; c < nv; ++c) {
+            const uint64_t ad = tc::sw128_kmajor_desc(a_0 + as * Sh::A_BYTES + c * Sh::A_SUB);
+            const uint64_t bd = tc::sw128_kmajor_desc(s_0 + ss * Sh::S_BYTES + c * Sh::B_SUB);
+            const int chunk = st * CH + c;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc::tc_mma(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
-          tc::tc_commit(aempty(as));  // this activation box has been read
-          tc::tc_commit(bempty(bs));  // and these converted weights
+            for (int kk = 0; kk < BK / UMMA_K; ++kk)
+              tc::tc_mma(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (chunk | kk) != 0 ? 1u : 0u);
+          }
+          tc::tc_commit(aempty(as));  // this stage's activations have been read
+          tc::tc_commit(empty(ss));   // and its decoded weights
+          if (++ss == NS) { ss = 0; sph ^= 1u; }
           if (++as == NA) { as = 0; aph ^= 1u; }
-          if (++bs == NB) { bs = 0; bph ^= 1u; }
         }
         if (!ok) break;
         tc::tc_commit(tfull(acc));
@@ -285,63 +304,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= CONV_WARP0 && warp < CONV_WARP0 + CONV_WARPS) {
     // ---------------------------------------------------------------- converters
-    // For the K step kb, 256 threads turn half (kb & 1) of the Q tile (chunks
-    // 4h..4h+3 of each 128-byte row, stored at chunk ^ (row & 7)) into the bf16
-    // tile: 16 codes -> two 16-byte chunks at (2c, 2c+1) ^ (row & 7). A thread
-    // owns rows r, r+64, r+128, r+192 with r & 7 = its lane & 7, so the 8 lanes
-    // of every shared-memory phase hit 8 different 16-byte bank groups, both
-    // when reading and when writing.
+    // For chunk g, 256 threads turn half (g & 1) of the Q tile (chunks 4h..4h+3
+    // of each 128-byte row, stored at chunk ^ (row & 7)) into the bf16 tile: 16
+    // codes -> two 16-byte chunks at (2c, 2c+1) ^ (row & 7). A thread owns rows
+    // r, r+64, r+128, r+192 with r & 7 = its lane & 7, so the 8 lanes of every
+    // shared-memory phase hit 8 different 16-byte bank groups, both when reading
+    // and when writing.
     const int ct = threadIdx.x - CONV_WARP0 * 32;
     const int r_lo = ct & 7, c4 = (ct >> 3) & 3, r_hi = ct >> 5;
     const int row0 = r_hi * 8 + r_lo;  // 0..63
     const int pos0 = ((2 * c4) ^ r_lo) << 4, pos1 = ((2 * c4 + 1) ^ r_lo) << 4;
     const uint32_t q_row = row0 * Sh::QK;
     const uint32_t b_row = r_hi * 1024 + r_lo * 128;
-    int qs = 0, bs = 0;
-    uint32_t qph = 0, bph = 0;
-    for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      bool ok = true;
-      for (int kb = 0; kb < kbs; ++kb) {
-        const int h = kb & 1;
-        // lane 0 waits (bounded); the others then observe the completed phase
-        // themselves (it cannot move on before this warp arrives), which gives
-        // each lane its own acquire for the TMA-written tile
+    const bool first = warp == CONV_WARP0;
+    int ss = 0, qs = 0, as = 0;
+    uint32_t sph = 0, qph = 0, aph = 0;
+    bool ok = true;
+    for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int st = 0; st < nst; ++st) {
+        // lane 0 waits (bounded) for the stage's slot to be free; __syncwarp
+        // then orders the other lanes' writes after it
         int w = 1;
-        if (lane == 0)
-          w = ((h != 0 || tc::wait_bounded(qfull(qs), qph, abort_flag, tmo)) &&
-               tc::wait_bounded(bempty(bs), bph ^ 1u, abort_flag, tmo))
-                  ? 1
-                  : 0;
+        if (lane == 0) w = tc::wait_bounded(empty(ss), sph ^ 1u, abort_flag, tmo) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        (void)tc::mbar_try_wait(qfull(qs), qph);
-        (void)tc::mbar_try_wait(bempty(bs), bph ^ 1u);
-        const uint8_t* q = q_base + qs * Sh::Q_BYTES + q_row + ((((4 * h + c4) ^ r_lo)) << 4);
-        uint8_t* b16 = b_base + bs * Sh::B16_BYTES + b_row;
-        uint4 v[4];
+        const int nv = min(CH, nck - st * CH);
+        uint8_t* const bst = s_base + ss * Sh::S_BYTES + b_row;
+        // all of this stage's codes are loaded before any is decoded (two
+        // chunks of independent work per thread hide the load latency)
+        uint4 v[CH][4];
+        for (int c = 0; c < nv; ++c) {
+          const int g = st * CH + c, h = g & 1;
+          if (h == 0) {
+            // lane 0 waits for the Q tile; the others then observe the completed
+            // phase themselves (it cannot move on before this warp releases it),
+            // which gives each lane its own acquire for the TMA-written bytes
+            w = 1;
+            if (lane == 0) w = tc::wait_bounded(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+            (void)tc::mbar_try_wait(qfull(qs), qph);
+          }
+          const uint8_t* q = q_base + qs * Sh::Q_BYTES + q_row + (((4 * h + c4) ^ r_lo) << 4);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(q + i * 64 * Sh::QK);
+          for (int i = 0; i < 4; ++i) v[c][i] = *reinterpret_cast<const uint4*>(q + i * 64 * Sh::QK);
+          if (h == 1 || g == nck - 1) {  // this Q tile is fully read: hand it back
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(qempty(qs));
+            if (++qs == NQ) { qs = 0; qph ^= 1u; }
+          }
+        }
+        if (!ok) break;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t o[8];
-          e4m3x4_to_bf16x4(v[i].x, o[0], o[1]);
-          e4m3x4_to_bf16x4(v[i].y, o[2], o[3]);
-          e4m3x4_to_bf16x4(v[i].z, o[4], o[5]);
-          e4m3x4_to_bf16x4(v[i].w, o[6], o[7]);
-          uint8_t* rowp = b16 + i * 8 * 1024;  // rows + 64 i
-          *reinterpret_cast<uint4*>(rowp + pos0) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(rowp + pos1) = make_uint4(o[4], o[5], o[6], o[7]);
+        for (int c = 0; c < CH; ++c) {
+          if (c >= nv) break;
+          uint8_t* b16 = bst + c * Sh::B_SUB;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t o[8];
+            e4m3x4_to_f16x4(v[c][i].x, o[0], o[1]);
+            e4m3x4_to_f16x4(v[c][i].y, o[2], o[3]);
+            e4m3x4_to_f16x4(v[c][i].z, o[4], o[5]);
+            e4m3x4_to_f16x4(v[c][i].w, o[6], o[7]);
+            uint8_t* rowp = b16 + i * 8 * 1024;  // rows + 64 i
+            *reinterpret_cast<uint4*>(rowp + pos0) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(rowp + pos1) = make_uint4(o[4], o[5], o[6], o[7]);
+          }
         }
         fence_async_shared();  // generic-proxy writes -> visible to the tensor cores
         __syncwarp();
-        const bool q_done = h == 1 || kb == kbs - 1;
         if (lane == 0) {
-          tc::mbar_arrive(bfull(bs));
-          if (q_done) tc::mbar_arrive(qempty(qs));
+          // the first converter warp also vouches for the activation boxes
+          if (first && !tc::wait_bounded(afull(as), aph, abort_flag, tmo)) ok = false;
+          tc::mbar_arrive(full(ss));
         }
-        if (q_done && ++qs == NQ) { qs = 0; qph ^= 1u; }
-        if (++bs == NB) { bs = 0; bph ^= 1u; }
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
+        if (++ss == NS) { ss = 0; sph ^= 1u; }
+        if (++as == NA) { as = 0; aph ^= 1u; }
       }
-      if (!ok) break;
     }
   } else {
     // ---------------------------------------------------------------- epilogue
@@ -378,7 +416,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const int col = col0 + qq * 8 + i;
                   h[i] = silu_f32(gv[qq * 8 + i] * sc0[col]) * (uv[qq * 8 + i] * sc1[col]);
                 }
-                st_v4(out + col0 + qq * 8, Vec16<__nv_bfloat16>::pack(h));
+                // H feeds the f16 x f16 down GEMM: stored as fp16
+                st_v4(out + col0 + qq * 8, make_uint4(f16x2_sat(h[0], h[1]), f16x2_sat(h[2], h[3]),
+                                                      f16x2_sat(h[4], h[5]), f16x2_sat(h[6], h[7])));
               }
             }
           }
@@ -467,9 +507,10 @@ __global__ void __launch_bounds__(256) dequantize_rows_fp8_kernel(const uint8_t*
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t lo, hi;
-      e4m3x4_to_bf16x4(in[j], lo, hi);
-      o[j] = make_float4(__uint_as_float(lo << 16) * s, __uint_as_float(lo & 0xFFFF0000u) * s,
-                         __uint_as_float(hi << 16) * s, __uint_as_float(hi & 0xFFFF0000u) * s);
+      e4m3x4_to_f16x4(in[j], lo, hi);
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+      o[j] = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
     }
   }
 }
