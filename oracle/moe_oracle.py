@@ -53,7 +53,7 @@ __all__ = [
     "GATE_RENORM", "GATE_RAW", "GATE_SIGMOID", "sigmoid_affinity", "balance_probs",
     "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
     "E4M3_MAX", "e4m3_round", "e4m3_encode", "e4m3_decode", "quantize_rows_fp8",
-    "dequantize_rows_fp8",
+    "dequantize_rows_fp8", "fake_quant_rows_fp8", "swiglu_ffn_w8a8",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
     "moe_param_count", "active_flops", "OracleResult",
 ]
@@ -310,7 +310,8 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
                 capacity_factor: float = 0.0, router_bias=None,
                 shared_weights: Optional[Sequence] = None,
                 rows: Optional[np.ndarray] = None, gate_mode: int = GATE_RENORM,
-                selection_bias=None, n_group: int = 1, topk_group: int = 1) -> OracleResult:
+                selection_bias=None, n_group: int = 1, topk_group: int = 1,
+                act_fp8: bool = False) -> OracleResult:
     """Forward pass of the routed MoE FFN layer, looping over experts.
 
     x: [T, d]; W_r: [E, d]; expert_weights(e) -> (W_g[e], W_u[e], W_d[e]);
@@ -325,6 +326,7 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
     the shared expert on every token with weight 1; the balance statistic.
     gate_mode, selection_bias, n_group and topk_group select the routing
     variants above (defaults: renormalised softmax top-k, no bias, no groups).
+    act_fp8: the routed experts run swiglu_ffn_w8a8 (R13) instead of swiglu_ffn.
     """
     T = x.shape[0]
     r = router_logits(x, W_r, router_bias)
@@ -357,7 +359,8 @@ def moe_forward(x, W_r, expert_weights: Callable[[int], Sequence], k: int,
             continue
         Wg, Wu, Wd = expert_weights(e)
         xe = xr[tok] if xr is not None else _f64(x[tok])
-        y[tok] += g[tok, slot][:, None] * swiglu_ffn(xe, Wg, Wu, Wd)
+        ffn = swiglu_ffn_w8a8 if act_fp8 else swiglu_ffn
+        y[tok] += g[tok, slot][:, None] * ffn(xe, Wg, Wu, Wd)
     if shared_weights is not None:
         xs = xr[rows] if xr is not None else _f64(x[rows])
         y[rows] += swiglu_ffn(xs, *shared_weights)
@@ -432,6 +435,30 @@ def quantize_rows_fp8(w):
 def dequantize_rows_fp8(codes, scales) -> np.ndarray:
     """The weights the layer computes with: code value times the row scale (fp64, exact)."""
     return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
+
+
+# R13 (FP8 on both operands): the GEMM inputs of a routed expert, the token
+# rows x and the hidden rows H, are quantised like the weights, one scale per
+# row (per token for x, per routed (token, expert) row for H); a GEMM then
+# computes with code * scale on both sides. Sources as above, plus Zero to
+# Frontier 13.1 "Why MoE" (the expert FFN is two GEMMs around SwiGLU).
+
+def fake_quant_rows_fp8(a) -> np.ndarray:
+    """Rows of `a` through the per-row E4M3 quantiser and back (fp64, exact)."""
+    codes, scales = quantize_rows_fp8(a)
+    return dequantize_rows_fp8(codes, scales)
+
+
+def swiglu_ffn_w8a8(x, W_g, W_u, W_d) -> np.ndarray:
+    """One SwiGLU expert with E4M3 activations (R13): x rows quantised per row,
+    the gate/up GEMM, SwiGLU in full precision, H rows quantised per row, the
+    down GEMM. W_g, W_u, W_d are the weights the layer computes with (for FP8
+    weights: code * scale)."""
+    xq = fake_quant_rows_fp8(_f64(x))
+    a = xq @ _f64(W_g).T
+    b = xq @ _f64(W_u).T
+    hq = fake_quant_rows_fp8(silu(a) * b)
+    return hq @ _f64(W_d).T
 
 
 # ----------------------------------------------------------------------------
