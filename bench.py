@@ -42,9 +42,10 @@ def parse_args():
     ap.add_argument("--workload", default="mixtral",
                     choices=["mixtral", "deepseek_v3", "switch_zipf", "decode", "tiny_fp32",
                              "mixtral_profile", "decode_profile"])
-    ap.add_argument("--weights", choices=["dtype", "fp8"], default="dtype",
-                    help="expert weights in the activation dtype, or E4M3 codes with per-row "
-                         "scales (quantised once by the library before timing)")
+    ap.add_argument("--weights", choices=["dtype", "fp8", "w8a8"], default="dtype",
+                    help="expert weights in the activation dtype; E4M3 codes with per-row "
+                         "scales (quantised once by the library before timing); or those and "
+                         "E4M3 activations inside the experts (W8A8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -229,7 +230,8 @@ def run_ours(args, rank, world, local_rank):
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     counts = torch.empty(w.E, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    fp8 = args.weights == "fp8"
+    fp8 = args.weights in ("fp8", "w8a8")
+    act_fp8 = args.weights == "w8a8"
     scales = None
     if fp8:  # one-off weight preparation, untimed
         parts = []
@@ -243,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
         forward(xs[i % R], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["W_shared"],
                 k=w.k, capacity_factor=w.capacity_factor, router_bias=inp["router_bias"],
                 d_s=w.d_s, workspace=ws, stream=stream, events=events, y=y, aux=aux,
-                counts=counts, weight_scales=scales)
+                counts=counts, weight_scales=scales, act_fp8=act_fp8)
 
     def barrier():
         if world > 1:
@@ -297,6 +299,8 @@ def run_ours(args, rank, world, local_rank):
     act_bytes = 2 * w.T * w.d * esz
     peaks, peaks_src = load_peaks()
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if act_fp8:  # E4M3 x E4M3: the bf16 figure times the nominal 4.5 / 2.25 ratio
+        tensor_peak *= 2.0
     hbm_peak = peaks["hbm_gbs"]
 
     ms_step = ms_max / args.steps
@@ -310,7 +314,8 @@ def run_ours(args, rank, world, local_rank):
     up_bound = "tensor" if flops_up / (tensor_peak * 1e12) >= bytes_up / (hbm_peak * 1e9) else "hbm"
     if up_bound == "tensor":
         achieved, peak, unit, work = flops_up / (k_up / 1e3) / 1e12, tensor_peak, "TFLOP/s", flops_up
-        peak_note = f"bf16_tflops_sustained (of {peaks_src})"
+        peak_note = (f"bf16_tflops_sustained x 2 (nominal e4m3/bf16 ratio; of {peaks_src})"
+                     if act_fp8 else f"bf16_tflops_sustained (of {peaks_src})")
     else:
         achieved, peak, unit, work = bytes_up / (k_up / 1e3) / 1e9, hbm_peak, "GB/s", bytes_up
         peak_note = f"hbm_gbs (of {peaks_src})"
@@ -319,10 +324,13 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "dtype": ("e4m3" if act_fp8 else ("bf16" if w.dtype == "bf16" else "f32")),
+        "data": "synthetic",
         "config": dict(config_of(w, "inputs larger than L2: %.2f GB of expert weights streamed "
                                     "per step; x rotates over %d batches" % (w_bytes / 1e9, R)),
-                       weights="e4m3 codes + fp32 row scales" if fp8 else w.dtype),
+                       weights="e4m3 codes + fp32 row scales" if fp8 else w.dtype,
+                       activations="e4m3 rows + fp32 row scales in the experts" if act_fp8
+                       else w.dtype),
         "roofline": {"bound": up_bound, "kernel": KERNEL_NAMES[4], "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": None,
                      "algorithmic_per_launch": work, "peak_source": peak_note},
@@ -333,7 +341,8 @@ def run_ours(args, rank, world, local_rank):
                   "dropped_fraction": O.dropped_fraction(cnt, C, w.T, w.k),
                   "aux": float(aux.cpu()[0])},
         "kernel_ms": {KERNEL_NAMES[j]: per_kernel[j] for j in range(MOE_NUM_KERNELS)},
-        "gpu_launches": MOE_NUM_KERNELS * args.steps * world,
+        # W8A8 adds the x and H quantisers to the 7 kernels of a step
+        "gpu_launches": (MOE_NUM_KERNELS + (2 if act_fp8 else 0)) * args.steps * world,
         "clocks": clk,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
     }
@@ -350,7 +359,9 @@ def run_ours(args, rank, world, local_rank):
         dims = _lib.make_dims(w.T, w.d, w.d_e, w.d_s,
                               _lib.MOE_BF16 if w.dtype == "bf16" else _lib.MOE_F32,
                               inp["router_bias"], ws.buf, nbytes, stream.cuda_stream,
-                              weight_format=_lib.MOE_WEIGHTS_FP8 if fp8 else _lib.MOE_WEIGHTS_DTYPE,
+                              weight_format=(_lib.MOE_WEIGHTS_FP8_W8A8 if act_fp8 else
+                                             _lib.MOE_WEIGHTS_FP8 if fp8 else
+                                             _lib.MOE_WEIGHTS_DTYPE),
                               weight_scales=scales)
 
         def e2e_call(i):

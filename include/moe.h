@@ -119,6 +119,16 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  */
 #define MOE_WEIGHTS_DTYPE 0
 #define MOE_WEIGHTS_FP8 1
+/*
+ * FP8 on both GEMM operands (W8A8): the weights as for MOE_WEIGHTS_FP8, and
+ * the routed experts' inputs quantised the same way, one fp32 scale per row:
+ * each token row of x (absmax over d) and each routed hidden row H (absmax
+ * over d_e) becomes E4M3 codes * scale. The expert GEMMs then run E4M3 x E4M3
+ * -> fp32 on the tensor cores, and both scales multiply the accumulator. This
+ * changes the numbers (activations carry 3 mantissa bits): it is a different
+ * layer from MOE_WEIGHTS_FP8, not a faster route to the same one.
+ */
+#define MOE_WEIGHTS_FP8_W8A8 2
 
 typedef struct {
   int64_t T;                 /* tokens in this call (0 allowed: empty batch) */
@@ -144,7 +154,9 @@ typedef struct {
   int32_t topk_group;        /* groups a token may pick from (1 <= topk_group <= n_group) */
   int32_t weight_format;     /* MOE_WEIGHTS_DTYPE (0): W_g, W_u, W_d in `dtype`;
                                 MOE_WEIGHTS_FP8 (1): E4M3 codes (uint8) with per-row scales,
-                                see moe_quantize_fp8 (bf16 activations, no shared expert) */
+                                see moe_quantize_fp8 (bf16 activations, no shared expert);
+                                MOE_WEIGHTS_FP8_W8A8 (2): the same weights, and E4M3
+                                activations inside the experts (see above) */
   const float* weight_scales; /* MOE_WEIGHTS_FP8: device fp32, the per-row scales of the three
                                  stacks one after another: W_g [E*d_e], W_u [E*d_e],
                                  W_d [E*d] (what moe_quantize_fp8 writes for each stack) */
@@ -219,6 +231,11 @@ typedef struct {
   size_t yrows;       /* dtype [rows_max, d]   gate-scaled expert outputs */
   int64_t rows_max;   /* rows reserved for the permuted buffers */
   int64_t capacity;   /* C, or -1 */
+  /* MOE_WEIGHTS_FP8_W8A8 only (0 otherwise); xp then holds E4M3 codes
+   * [rows_max, d] (row stride d bytes) */
+  size_t xscale;      /* fp32 [rows_max]       scale of each permuted x row */
+  size_t hq;          /* uint8 [rows_max, d_e] E4M3 codes of the hidden rows */
+  size_t hscale;      /* fp32 [rows_max]       scale of each hidden row */
 } moe_workspace_layout_t;
 
 MOE_API moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capacity_factor,

@@ -46,6 +46,7 @@ import math
 from typing import Callable, Optional, Sequence
 
 import numpy as np
+import torch
 
 __all__ = [
     "router_logits", "softmax_all", "top_k", "gates_softmax_topk", "gates_renormalised",
@@ -53,7 +54,7 @@ __all__ = [
     "GATE_RENORM", "GATE_RAW", "GATE_SIGMOID", "sigmoid_affinity", "balance_probs",
     "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
     "E4M3_MAX", "e4m3_round", "e4m3_encode", "e4m3_decode", "quantize_rows_fp8",
-    "dequantize_rows_fp8", "fake_quant_rows_fp8", "swiglu_ffn_w8a8",
+    "dequantize_rows_fp8", "fake_quant_rows_fp8", "round_bf16", "swiglu_ffn_w8a8",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
     "moe_param_count", "active_flops", "OracleResult",
 ]
@@ -449,15 +450,23 @@ def fake_quant_rows_fp8(a) -> np.ndarray:
     return dequantize_rows_fp8(codes, scales)
 
 
+def round_bf16(a) -> np.ndarray:
+    """fp64 -> fp32 -> bf16, each step round-to-nearest-even (torch's casts), as fp64."""
+    t = torch.tensor(np.asarray(a, dtype=np.float64), dtype=torch.float32)
+    return t.to(torch.bfloat16).to(torch.float64).numpy()
+
+
 def swiglu_ffn_w8a8(x, W_g, W_u, W_d) -> np.ndarray:
     """One SwiGLU expert with E4M3 activations (R13): x rows quantised per row,
     the gate/up GEMM, SwiGLU in full precision, H rows quantised per row, the
     down GEMM. W_g, W_u, W_d are the weights the layer computes with (for FP8
-    weights: code * scale)."""
+    weights: code * scale). R13b: H is held in bf16 before its quantisation (the
+    precision the layer stores it in), so that both sides decide H's codes from
+    the same values."""
     xq = fake_quant_rows_fp8(_f64(x))
     a = xq @ _f64(W_g).T
     b = xq @ _f64(W_u).T
-    hq = fake_quant_rows_fp8(silu(a) * b)
+    hq = fake_quant_rows_fp8(round_bf16(silu(a) * b))
     return hq @ _f64(W_d).T
 
 

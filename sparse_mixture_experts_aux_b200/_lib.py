@@ -22,7 +22,7 @@ MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_GATE_RENORM, MOE_GATE_RAW, MOE_GATE_SIGMOID = 0, 1, 2
-MOE_WEIGHTS_DTYPE, MOE_WEIGHTS_FP8 = 0, 1
+MOE_WEIGHTS_DTYPE, MOE_WEIGHTS_FP8, MOE_WEIGHTS_FP8_W8A8 = 0, 1, 2
 MOE_NUM_KERNELS = 7
 KERNEL_NAMES = ("router_logits", "route", "scan", "scatter", "gate_up_swiglu", "down_scale", "combine")
 
@@ -66,6 +66,9 @@ class moe_workspace_layout_t(ctypes.Structure):
         ("yrows", ctypes.c_size_t),
         ("rows_max", ctypes.c_int64),
         ("capacity", ctypes.c_int64),
+        ("xscale", ctypes.c_size_t),
+        ("hq", ctypes.c_size_t),
+        ("hscale", ctypes.c_size_t),
     ]
 
 

@@ -37,7 +37,11 @@ struct Plan {
   bool router_narrow;  // few experts, many tokens: warp-per-token-group router kernel
   int64_t rows_max;
   size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
-      o_tile_start, o_pair_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys, total;
+      o_tile_start, o_pair_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys,
+      // E4M3 activations (MOE_WEIGHTS_FP8_W8A8): x codes and scales per token,
+      // scales of the permuted x rows, H codes and scales per permuted row
+      o_xq, o_sx, o_xsc, o_hq, o_hsc, total;
+  bool w8a8;
 };
 
 int64_t capacity_of(int64_t T, int E, int k, float cf) {
@@ -67,9 +71,10 @@ moe_status check_dims(const moe_dims* dims, int E, int k, float cf) {
   if (dims->T * static_cast<int64_t>(k) >= (int64_t(1) << 31) ||
       dims->T * static_cast<int64_t>(E) >= (int64_t(1) << 40))
     return MOE_ERR_UNSUPPORTED;
-  if (dims->weight_format != MOE_WEIGHTS_DTYPE && dims->weight_format != MOE_WEIGHTS_FP8)
+  if (dims->weight_format != MOE_WEIGHTS_DTYPE && dims->weight_format != MOE_WEIGHTS_FP8 &&
+      dims->weight_format != MOE_WEIGHTS_FP8_W8A8)
     return MOE_ERR_INVALID_ARG;
-  if (dims->weight_format == MOE_WEIGHTS_FP8 && (dims->dtype != MOE_BF16 || dims->d_s != 0))
+  if (dims->weight_format != MOE_WEIGHTS_DTYPE && (dims->dtype != MOE_BF16 || dims->d_s != 0))
     return MOE_ERR_UNSUPPORTED;
   const int mult = dims->dtype == MOE_BF16 ? 64 : 32;
   if (dims->d % mult || dims->d_e % mult || dims->d_s % mult) return MOE_ERR_UNSUPPORTED;
@@ -117,6 +122,12 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   p.o_yrows = take(R * p.d * p.esz);
   p.o_hs = take(p.ds ? T * p.ds * p.esz : 0);
   p.o_ys = take(p.ds ? T * p.d * p.esz : 0);
+  p.w8a8 = dims->weight_format == MOE_WEIGHTS_FP8_W8A8;
+  p.o_xq = take(p.w8a8 ? T * p.d : 0);
+  p.o_sx = take(p.w8a8 ? T * 4 : 0);
+  p.o_xsc = take(p.w8a8 ? R * 4 : 0);
+  p.o_hq = take(p.w8a8 ? R * p.de : 0);
+  p.o_hsc = take(p.w8a8 ? R * 4 : 0);
   p.total = off;
   return p;
 }
@@ -139,9 +150,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-template <int EPI, int AR>
+template <int EPI, int AR, bool Q8 = false>
 bool tc_attr() {
-  return cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<EPI, AR>,
+  return cudaFuncSetAttribute(moe::tc::tc_grouped_gemm_kernel<EPI, AR, Q8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               moe::tc::TcShape<AR>::SMEM_BYTES) == cudaSuccess;
 }
@@ -166,18 +177,21 @@ void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
         <<<grid, NUM_THREADS, F8Shape<128>::SMEM_BYTES, st>>>(maps, fp);
 }
 
-// 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32).
-template <int EPI>
+// 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32);
+// Q8: E4M3 operands.
+template <int EPI, bool Q8 = false>
 void launch_tc(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
                const moe::tc::TcParams& tp) {
   using namespace moe::tc;
   if (ar == 32)
-    tc_grouped_gemm_kernel<EPI, 32><<<grid, NUM_THREADS, TcShape<32>::SMEM_BYTES, st>>>(maps, tp);
+    tc_grouped_gemm_kernel<EPI, 32, Q8>
+        <<<grid, NUM_THREADS, TcShape<32>::SMEM_BYTES, st>>>(maps, tp);
   else if (ar == 64)
-    tc_grouped_gemm_kernel<EPI, 64><<<grid, NUM_THREADS, TcShape<64>::SMEM_BYTES, st>>>(maps, tp);
+    tc_grouped_gemm_kernel<EPI, 64, Q8>
+        <<<grid, NUM_THREADS, TcShape<64>::SMEM_BYTES, st>>>(maps, tp);
   else
-    tc_grouped_gemm_kernel<EPI, 128><<<grid, NUM_THREADS, TcShape<128>::SMEM_BYTES, st>>>(maps,
-                                                                                           tp);
+    tc_grouped_gemm_kernel<EPI, 128, Q8>
+        <<<grid, NUM_THREADS, TcShape<128>::SMEM_BYTES, st>>>(maps, tp);
 }
 
 template <int EPI>
@@ -230,6 +244,11 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
     if (!tc_attr<moe::tc::EPI_SWIGLU_TC, 128>() || !tc_attr<moe::tc::EPI_SCALE_TC, 128>() ||
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64>() ||
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 32>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32>())
+      return MOE_ERR_CUDA;
+    if (!tc_attr<moe::tc::EPI_SWIGLU_TC, 128, true>() ||
+        !tc_attr<moe::tc::EPI_SCALE_TC, 128, true>() ||
+        !tc_attr<moe::tc::EPI_SWIGLU_TC, 64, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64, true>() ||
+        !tc_attr<moe::tc::EPI_SWIGLU_TC, 32, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32, true>())
       return MOE_ERR_CUDA;
     if (!f8_attr<moe::tc::EPI_SWIGLU_TC, 128>() || !f8_attr<moe::tc::EPI_SCALE_TC, 128>() ||
         !f8_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !f8_attr<moe::tc::EPI_SCALE_TC, 64>() ||
@@ -407,11 +426,23 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   {
     const int nvec = static_cast<int>(static_cast<size_t>(P.d) * sizeof(TX) / 16);
     dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
-    if (dims->weight_format == MOE_WEIGHTS_FP8)  // the FP8-weight GEMMs read fp16 rows
+    if (P.w8a8) {
+      // E4M3 activations: quantise each token row once (scale per token), then
+      // scatter the code rows and carry each row's scale to its slots
+      uint8_t* xq = ws + P.o_xq;
+      float* sx = reinterpret_cast<float*>(ws + P.o_sx);
+      moe::tcf8::quantize_rows_fp8_kernel<TX><<<static_cast<unsigned>(T < 8192 ? T : 8192), 256,
+                                                 0, st>>>(x, T, P.d, xq, sx);
+      const int qvec = P.d / 16;
+      dim3 qgrid((T + 7) / 8, (qvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
+      moe::scatter_kernel<uint8_t><<<qgrid, 256, 0, st>>>(
+          xq, P.d, T, P.k, P.E, P.C, idx, gate, lrank, base, tile_start, slot, rowgate,
+          reinterpret_cast<uint8_t*>(xp), sx, reinterpret_cast<float*>(ws + P.o_xsc));
+    } else if (dims->weight_format == MOE_WEIGHTS_FP8) {  // the FP8-weight GEMMs read fp16 rows
       moe::scatter_kernel<TX, true><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate,
                                                           lrank, base, tile_start, slot, rowgate,
                                                           xp);
-    else
+    } else
       moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
                                                     base, tile_start, slot, rowgate, xp);
   }
@@ -443,7 +474,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   if (dims->router_bias != nullptr && !aligned(dims->router_bias, 16)) return MOE_ERR_INVALID_ARG;
   if (dims->selection_bias != nullptr && !aligned(dims->selection_bias, 16))
     return MOE_ERR_INVALID_ARG;
-  if (dims->weight_format == MOE_WEIGHTS_FP8 &&
+  if (dims->weight_format != MOE_WEIGHTS_DTYPE &&
       (dims->weight_scales == nullptr || !aligned(dims->weight_scales, 4)))
     return MOE_ERR_INVALID_ARG;
 
@@ -479,7 +510,52 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     const size_t sh_n = static_cast<size_t>(P.ds) * P.d;
     const int ng = P.ds ? 2 : 1;
 
-    if (dims->weight_format == MOE_WEIGHTS_FP8) {
+    if (P.w8a8) {
+      // E4M3 x E4M3 (kind::f8f6f4) on the 1-CTA kernels; H is quantised per row
+      // between the two GEMMs
+      const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
+      const float* sc = dims->weight_scales;
+      const size_t gsz = static_cast<size_t>(E) * P.de;
+      uint8_t* hq = ws + P.o_hq;
+      float* xsc = reinterpret_cast<float*>(ws + P.o_xsc);
+      float* hsc = reinterpret_cast<float*>(ws + P.o_hsc);
+      constexpr int K8 = 128;  // codes per K step
+      moe::tc::TcMaps up, dn;
+      memset(&up, 0, sizeof(up));
+      memset(&dn, 0, sizeof(dn));
+      // the code rows are described to TMA as 16-bit elements (2 codes each),
+      // with the same boxes as the bf16 path: 128-byte lines, 128-byte swizzle
+      const bool ok = encode_map(&up.a[0], xp, P.d / 2, P.rows_max, 1, arows, 2) &&
+                      encode_map(&up.b0[0], W_g, P.d / 2, P.de, E, moe::tc::BN / 2, 3) &&
+                      encode_map(&up.b1[0], W_u, P.d / 2, P.de, E, moe::tc::BN / 2, 3) &&
+                      encode_map(&dn.a[0], hq, P.de / 2, P.rows_max, 1, arows, 2) &&
+                      encode_map(&dn.b0[0], W_d, P.de / 2, P.d, E, moe::tc::BN, 3);
+      if (!ok) return MOE_ERR_CUDA;
+      dn.b1[0] = dn.b0[0];
+      moe::tc::TcParams tu{};
+      tu.num_groups = 1;
+      tu.timeout_ns = wait_tmo;
+      tu.drain_timeout_ns = kDrainTimeoutNs;
+      tu.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+                 (P.d + K8 - 1) / K8, P.de, h, nullptr, xsc, sc, sc + gsz, P.de};
+      moe::tc::TcParams td{};
+      td.num_groups = 1;
+      td.timeout_ns = wait_tmo;
+      td.drain_timeout_ns = kDrainTimeoutNs;
+      td.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, (P.de + K8 - 1) / K8,
+                 P.d, yrows, rowgate, hsc, sc + 2 * gsz, sc + 2 * gsz, P.d};
+      tm.at(8);
+      launch_tc<moe::tc::EPI_SWIGLU_TC, true>(arows, num_sms, st, up, tu);
+      tm.at(9);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+      tm.at(10);
+      moe::tcf8::quantize_rows_fp8_kernel<bf16>
+          <<<static_cast<unsigned>(P.rows_max < 8192 ? P.rows_max : 8192), 256, 0, st>>>(
+              h, P.rows_max, P.de, hq, hsc, tile_start + E);
+      launch_tc<moe::tc::EPI_SCALE_TC, true>(arows, num_sms, st, dn, td);
+      tm.at(11);
+      if (launched() != MOE_OK) return MOE_ERR_CUDA;
+    } else if (dims->weight_format == MOE_WEIGHTS_FP8) {
       // FP8 expert weights: 1-CTA kernels that dequantise the weight tiles on chip
       const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
       const float* sc = dims->weight_scales;
@@ -718,6 +794,9 @@ moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capaci
   out->yrows = P.o_yrows;
   out->rows_max = P.rows_max;
   out->capacity = P.C;
+  out->xscale = P.o_xsc;
+  out->hq = P.o_hq;
+  out->hscale = P.o_hsc;
   return MOE_OK;
 }
 

@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ gate,
     const int32_t* __restrict__ lrank, const int32_t* __restrict__ base,
     const int32_t* __restrict__ tile_start, int32_t* __restrict__ slot_pos,
-    float* __restrict__ row_gate, TX* __restrict__ xp) {
+    float* __restrict__ row_gate, TX* __restrict__ xp,
+    const float* __restrict__ scale_in = nullptr, float* __restrict__ scale_out = nullptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;  // warp-uniform
@@ -61,7 +62,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int rank = base[(size_t)(t / ROUTE_CHUNK) * E + e] + lrank[a];
     if (C < 0 || (int64_t)rank < C) mypos = tile_start[e] * ROW_TILE + rank;
     if (blockIdx.y == 0) {
-      if (mypos >= 0) row_gate[mypos] = gate[a];
+      if (mypos >= 0) {
+        row_gate[mypos] = gate[a];
+        if (scale_out != nullptr) scale_out[mypos] = scale_in[t];  // E4M3 rows' scales
+      }
       slot_pos[a] = mypos;
     }
   }

@@ -468,7 +468,11 @@ template <typename TW>
 __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const TW* __restrict__ w,
                                                                 int64_t rows, int cols,
                                                                 uint8_t* __restrict__ codes,
-                                                                float* __restrict__ scales) {
+                                                                float* __restrict__ scales,
+                                                                const int32_t* tiles_end = nullptr) {
+  // tiles_end (optional): rows beyond *tiles_end * 128 are left alone (the
+  // permuted buffers' unused tail)
+  if (tiles_end != nullptr) rows = min(rows, (int64_t)(*tiles_end) * ROW_TILE);
   __shared__ float red[8];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const TW* wr = w + r * cols;

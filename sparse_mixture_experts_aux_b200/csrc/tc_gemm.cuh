@@ -72,6 +72,12 @@ struct TcGroup {
   int N;                      // output columns
   void* out;                  // bf16 [rows, N]
   const float* row_scale;     // scale epilogue: factor per row; NULL = 1
+  // E4M3 operands (Q8 kernels only): A row scales, B row scales of the
+  // output columns (gate/up: b_scale0 gate, b_scale1 up), floats per expert
+  const float* a_scale;
+  const float* b_scale0;
+  const float* b_scale1;
+  int64_t b_scale_stride;
 };
 
 struct TcParams {
@@ -208,6 +214,19 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
+// The same with E4M3 operands (kind::f8f6f4): 32 codes of K per instruction,
+// so a 128-byte shared-memory row is 128 codes and the descriptors advance
+// exactly as for bf16 (+32 bytes per instruction).
+__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
 // Load 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one row per
 // thread) and wait for them in the same asm block, so that no use of the
 // registers can be scheduled before the wait.
@@ -247,6 +266,10 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+// kind::f8f6f4 with A and B E4M3 (format 0), D fp32, both K-major.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 struct TileInfo {
@@ -290,9 +313,14 @@ __device__ __forceinline__ TileInfo decode_tile(long long tile, long long tiles0
   return ti;
 }
 
-template <int EPI, int AR>
+// Q8: A and B are E4M3 codes (tensor maps over 16-bit elements, 2 codes each,
+// so a K step is the same 128-byte line as in bf16: 128 codes), and the
+// epilogue multiplies each accumulator by the A row's and the B column's
+// scales before its own arithmetic.
+template <int EPI, int AR, bool Q8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  constexpr int KX = BK;  // TMA x-coordinate units (16-bit elements) per K step
   constexpr int STAGES = TcShape<AR>::STAGES;
   constexpr int A_BYTES = TcShape<AR>::A_BYTES;
   constexpr int STAGE_BYTES = TcShape<AR>::STAGE_BYTES;
@@ -368,12 +396,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full_bar(stage);
           mbar_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(sa, &maps.a[ti.g], fb, kb * BK, ti.row0);
+          tma_load_2d(sa, &maps.a[ti.g], fb, kb * KX, ti.row0);
           if (EPI == EPI_SWIGLU_TC) {
-            tma_load_3d(sb, &maps.b0[ti.g], fb, kb * BK, ti.nb * (BN / 2), ti.e);
-            tma_load_3d(sb + B_BYTES / 2, &maps.b1[ti.g], fb, kb * BK, ti.nb * (BN / 2), ti.e);
+            tma_load_3d(sb, &maps.b0[ti.g], fb, kb * KX, ti.nb * (BN / 2), ti.e);
+            tma_load_3d(sb + B_BYTES / 2, &maps.b1[ti.g], fb, kb * KX, ti.nb * (BN / 2), ti.e);
           } else {
-            tma_load_3d(sb, &maps.b0[ti.g], fb, kb * BK, ti.nb * BN, ti.e);
+            tma_load_3d(sb, &maps.b0[ti.g], fb, kb * KX, ti.nb * BN, ti.e);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -388,7 +416,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = make_idesc(BM, BN);
+      constexpr uint32_t IDESC = Q8 ? make_idesc_e4m3(BM, BN) : make_idesc(BM, BN);
       int stage = 0;
       uint32_t phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
@@ -407,7 +435,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             // +32 bytes per K step = +2 in the descriptor's address field
-            tc_mma(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            if (Q8)
+              tc_mma_e4m3(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -438,6 +469,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tb = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
       if (quad * 32 < AR) {
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.N;
+      // E4M3 operands: the A row's scale, and the B scales of this expert
+      const float ars = (Q8 && row_ok) ? g.a_scale[row] : 1.f;
+      const float* bs0 = Q8 ? g.b_scale0 + (int64_t)ti.e * g.b_scale_stride : nullptr;
+      const float* bs1 = Q8 ? g.b_scale1 + (int64_t)ti.e * g.b_scale_stride : nullptr;
       if (EPI == EPI_SWIGLU_TC) {
 #pragma unroll 1
         for (int c = 0; c < (BN / 2) / 32; ++c) {
@@ -451,13 +486,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int q = 0; q < 4; ++q) {
               float h[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) h[i] = silu_f32(gv[q * 8 + i]) * uv[q * 8 + i];
+              for (int i = 0; i < 8; ++i) {
+                float a = gv[q * 8 + i], b = uv[q * 8 + i];
+                if (Q8) {
+                  const int col = col0 + q * 8 + i;
+                  a *= ars * bs0[col];
+                  b *= ars * bs1[col];
+                }
+                h[i] = silu_f32(a) * b;
+              }
               st_v4(out + col0 + q * 8, Vec16<__nv_bfloat16>::pack(h));
             }
           }
         }
       } else {
-        const float sc = (row_ok && g.row_scale != nullptr) ? g.row_scale[row] : 1.f;
+        const float sc = ((row_ok && g.row_scale != nullptr) ? g.row_scale[row] : 1.f) * ars;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
@@ -469,7 +512,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int q = 0; q < 4; ++q) {
               float h[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) h[i] = sc * v[q * 8 + i];
+              for (int i = 0; i < 8; ++i)
+                h[i] = Q8 ? sc * (v[q * 8 + i] * bs0[col0 + q * 8 + i]) : sc * v[q * 8 + i];
               st_v4(out + col0 + q * 8, Vec16<__nv_bfloat16>::pack(h));
             }
           }

@@ -31,11 +31,14 @@ class Workspace:
 
 
 def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, stream, events,
-              wait_timeout_ns: int = 0, routing: Optional[dict] = None, weight_scales=None):
+              wait_timeout_ns: int = 0, routing: Optional[dict] = None, weight_scales=None,
+              act_fp8: bool = False):
     T, d = x.shape
     d_e = W_g.shape[1]
     routing = routing or {}
-    fp8 = W_g.dtype == torch.uint8
+    fmt = _lib.MOE_WEIGHTS_DTYPE
+    if W_g.dtype == torch.uint8:
+        fmt = _lib.MOE_WEIGHTS_FP8_W8A8 if act_fp8 else _lib.MOE_WEIGHTS_FP8
     return _lib.make_dims(T, d, d_e, d_s, dtype_code(x.dtype), router_bias, ws,
                           ws.numel() if ws is not None else 0, stream, events,
                           wait_timeout_ns=wait_timeout_ns,
@@ -43,8 +46,7 @@ def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, str
                           selection_bias=routing.get("selection_bias"),
                           n_group=routing.get("n_group", 0),
                           topk_group=routing.get("topk_group", 0),
-                          weight_format=_lib.MOE_WEIGHTS_FP8 if fp8 else _lib.MOE_WEIGHTS_DTYPE,
-                          weight_scales=weight_scales)
+                          weight_format=fmt, weight_scales=weight_scales)
 
 
 def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Tensor,
@@ -54,13 +56,16 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
             y: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
             counts: Optional[torch.Tensor] = None, wait_timeout_ns: int = 0,
             gate_mode: int = 0, selection_bias: Optional[torch.Tensor] = None,
-            n_group: int = 0, topk_group: int = 0, weight_scales: Optional[torch.Tensor] = None):
+            n_group: int = 0, topk_group: int = 0, weight_scales: Optional[torch.Tensor] = None,
+            act_fp8: bool = False):
     """Run the routed MoE FFN layer; returns (y, aux[1] fp32, counts[E] int32) on x's device.
 
     Shapes: x [T, d]; W_r [E, d] fp32; W_g, W_u [E, d_e, d]; W_d [E, d, d_e];
     W_shared packed [gate d_s*d | up d_s*d | down d*d_s] when d_s > 0.
     FP8 expert weights: W_g, W_u, W_d as uint8 E4M3 codes (quantize_fp8) and
     weight_scales = their per-row scales concatenated [W_g | W_u | W_d] (bf16 x).
+    act_fp8 (with FP8 weights): E4M3 activations inside the experts as well
+    (MOE_WEIGHTS_FP8_W8A8 in include/moe.h).
     wait_timeout_ns: limit of the GEMM kernels' device-side waits (0 = library default).
     gate_mode / selection_bias / n_group / topk_group: routing variants (include/moe.h).
     """
@@ -81,14 +86,16 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
     if W_g.dtype == torch.uint8:
         if weight_scales is None or not weight_scales.is_cuda or weight_scales.dtype != torch.float32:
             raise RuntimeError("FP8 weights need weight_scales: a CUDA fp32 tensor")
+    elif act_fp8:
+        raise RuntimeError("act_fp8 needs FP8 (uint8) weights")
     probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events, routing=routing,
-                      weight_scales=weight_scales)
+                      weight_scales=weight_scales, act_fp8=act_fp8)
     nbytes = _lib.moe_workspace_size(probe, E, k, capacity_factor)
     if nbytes == 0:
         raise _lib.MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
     ws = workspace.get(nbytes, dev)
     dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns, routing,
-                     weight_scales)
+                     weight_scales, act_fp8)
     y = torch.empty_like(x) if y is None else y
     aux = torch.empty(1, dtype=torch.float32, device=dev) if aux is None else aux
     counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
@@ -125,10 +132,11 @@ def dequantize_fp8(codes: torch.Tensor, scales: torch.Tensor, stream=None) -> to
 
 
 def routing_views(ws: torch.Tensor, x: torch.Tensor, W_g: torch.Tensor, E: int, k: int,
-                  capacity_factor: float = 0.0, d_s: int = 0) -> dict:
-    """Views of the routing results moe_forward left in workspace `ws`."""
+                  capacity_factor: float = 0.0, d_s: int = 0, act_fp8: bool = False) -> dict:
+    """Views of the routing results moe_forward left in workspace `ws` (with
+    act_fp8 and FP8 weights, also the E4M3 activation rows and their scales)."""
     T, d = x.shape
-    dims = _dims_for(x, W_g, d_s, None, ws, 0, None)
+    dims = _dims_for(x, W_g, d_s, None, ws, 0, None, act_fp8=act_fp8)
     L = _lib.moe_workspace_layout(dims, E, k, capacity_factor)
     b = ws
 
@@ -148,4 +156,8 @@ def routing_views(ws: torch.Tensor, x: torch.Tensor, W_g: torch.Tensor, E: int, 
         h=view(L.h, L.rows_max * d_e, x.dtype).view(L.rows_max, d_e),
         yrows=view(L.yrows, L.rows_max * d, x.dtype).view(L.rows_max, d),
         rows_max=L.rows_max, capacity=L.capacity,
+        **(dict(xq=view(L.xp, L.rows_max * d, torch.uint8).view(L.rows_max, d),
+                xscale=view(L.xscale, L.rows_max, torch.float32),
+                hq=view(L.hq, L.rows_max * d_e, torch.uint8).view(L.rows_max, d_e),
+                hscale=view(L.hscale, L.rows_max, torch.float32)) if act_fp8 else {}),
     )

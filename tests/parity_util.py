@@ -15,9 +15,10 @@ GATE_TOL = 1e-6      # absolute, on gates
 Y_TOL = {"f32": 1e-4, "bf16": 2e-2}  # max|err| <= tol * max(1, |ref|)
 
 
-def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None, fp8: dict | None = None):
+def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None, fp8: dict | None = None,
+            act_fp8: bool = False):
     """fp8: E4M3 codes W_g, W_u, W_d and weight_scales (device) to use instead of
-    the dtype weights in `inp`."""
+    the dtype weights in `inp`; act_fp8: E4M3 activations too (W8A8)."""
     ws = ws or Workspace()
     src = fp8 if fp8 is not None else inp
     y, aux, counts = forward(inp["x"], inp["W_r"], src["W_g"], src["W_u"], src["W_d"],
@@ -25,14 +26,17 @@ def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None, fp8: dict | Non
                              router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws,
                              gate_mode=w.gate_mode, selection_bias=inp.get("selection_bias"),
                              n_group=w.n_group, topk_group=w.topk_group,
-                             weight_scales=fp8["weight_scales"] if fp8 is not None else None)
+                             weight_scales=fp8["weight_scales"] if fp8 is not None else None,
+                             act_fp8=act_fp8)
     torch.cuda.synchronize()
     assert moe_get_device_status() == 0, "a device-side wait timed out"
-    views = routing_views(ws.buf, inp["x"], inp["W_g"], w.E, w.k, w.capacity_factor, w.d_s)
+    views = routing_views(ws.buf, inp["x"], src["W_g"], w.E, w.k, w.capacity_factor, w.d_s,
+                          act_fp8=act_fp8)
     return y, aux, counts, views
 
 
-def run_oracle(w: Workload, inp: dict, rows=None, fp8: dict | None = None) -> O.OracleResult:
+def run_oracle(w: Workload, inp: dict, rows=None, fp8: dict | None = None,
+               act_fp8: bool = False) -> O.OracleResult:
     """fp8: as in run_gpu; the oracle then computes with code * scale (its own
     dequantisation, fp64)."""
     x = inp["x"].cpu()
@@ -55,7 +59,8 @@ def run_oracle(w: Workload, inp: dict, rows=None, fp8: dict | None = None) -> O.
     return O.moe_forward(x, inp["W_r"].cpu(), expert, w.k, layer_capacity_factor(w), bias, shared,
                          rows, gate_mode=w.gate_mode,
                          selection_bias=sel.cpu() if sel is not None else None,
-                         n_group=max(w.n_group, 1), topk_group=max(w.topk_group, 1))
+                         n_group=max(w.n_group, 1), topk_group=max(w.topk_group, 1),
+                         act_fp8=act_fp8)
 
 
 def layer_capacity_factor(w: Workload) -> float:

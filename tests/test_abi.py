@@ -107,6 +107,8 @@ def test_workspace_size_and_layout(lib):
     (8, 2, dict(weight_format=5), _lib.MOE_ERR_INVALID_ARG),
     (8, 2, dict(weight_format=1, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),  # FP8: bf16 x
     (8, 2, dict(weight_format=1, d_s=128), _lib.MOE_ERR_UNSUPPORTED),  # FP8: no shared expert
+    (8, 2, dict(weight_format=2, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),  # W8A8: bf16 x
+    (8, 2, dict(weight_format=3), _lib.MOE_ERR_INVALID_ARG),
 ])
 def test_forward_rejects_bad_shapes_on_host(lib, E, k, kw, want):
     d = _dims(**kw)
@@ -164,6 +166,15 @@ def test_fp8_weights_validated_on_host(lib):
     assert fwd(_dims(weight_format=1, weight_scales=g + 2)) == _lib.MOE_ERR_INVALID_ARG
     assert _lib.moe_workspace_size(_dims(weight_format=1, weight_scales=g), 8, 2, 0.0) > 0
     assert fwd(_dims(weight_format=1, weight_scales=g)) == _lib.MOE_ERR_WORKSPACE  # valid
+    assert fwd(_dims(weight_format=2, weight_scales=g)) == _lib.MOE_ERR_WORKSPACE  # valid
+    assert fwd(_dims(weight_format=2)) == _lib.MOE_ERR_INVALID_ARG  # scales missing
+    # W8A8 needs more workspace (activation codes and scales) and reports where they are
+    n1 = _lib.moe_workspace_size(_dims(weight_format=1), 8, 2, 0.0)
+    n2 = _lib.moe_workspace_size(_dims(weight_format=2), 8, 2, 0.0)
+    assert n2 > n1
+    L = _lib.moe_workspace_layout(_dims(weight_format=2), 8, 2, 0.0)
+    assert 0 < L.xscale < n2 and 0 < L.hq < n2 and 0 < L.hscale < n2
+    assert L.hq + L.rows_max * 256 <= n2
     # quantiser and dequantiser: argument checks on the host, nothing launched
     for args in [(0, 1, 4, 64, g, g), (g, 1, 4, 64, 0, g), (g, 1, 4, 64, g, 0), (g, 1, 4, 24, g, g),
                  (g, 1, -1, 64, g, g), (g, 9, 4, 64, g, g), (g, 1, 4, 0, g, g)]:
