@@ -256,8 +256,9 @@ MOE_API const char* moe_status_string(moe_status s);
  * routed expert stack, W_g [E, d_e, d] is rows = E * d_e, cols = d (likewise
  * W_u), and W_d [E, d, d_e] is rows = E * d, cols = d_e. Writing the three
  * stacks' scales one after another gives moe_dims.weight_scales. Returns
- * MOE_ERR_INVALID_ARG for null pointers, cols not a multiple of 16, rows < 0
- * or a bad dtype (nothing is launched), MOE_ERR_CUDA on launch failure.
+ * MOE_ERR_INVALID_ARG for null pointers, cols not a multiple of 16, rows < 0,
+ * a bad dtype, or w / codes not 16-byte aligned (nothing is launched),
+ * MOE_ERR_CUDA on launch failure.
  */
 MOE_API moe_status moe_quantize_fp8(const void* w, int32_t dtype, int64_t rows, int32_t cols,
                                     uint8_t* codes, float* scales, void* stream);

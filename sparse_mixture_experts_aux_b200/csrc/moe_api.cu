@@ -551,7 +551,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tm.at(10);
       moe::tcf8::quantize_rows_fp8_kernel<bf16>
           <<<static_cast<unsigned>(P.rows_max < 8192 ? P.rows_max : 8192), 256, 0, st>>>(
-              h, P.rows_max, P.de, hq, hsc, tile_start + E);
+              h, P.rows_max, P.de, hq, hsc, tile_start, counts, E, P.C);
       launch_tc<moe::tc::EPI_SCALE_TC, true>(arows, num_sms, st, dn, td);
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
@@ -862,7 +862,8 @@ const char* moe_status_string(moe_status s) {
 moe_status moe_quantize_fp8(const void* w, int32_t dtype, int64_t rows, int32_t cols,
                             uint8_t* codes, float* scales, void* stream) {
   if (w == nullptr || codes == nullptr || scales == nullptr || rows < 0 || cols < 1 ||
-      cols % 16 != 0 || (dtype != MOE_BF16 && dtype != MOE_F32) || !aligned(scales, 4))
+      cols % 16 != 0 || (dtype != MOE_BF16 && dtype != MOE_F32) || !aligned(scales, 4) ||
+      !aligned(w, 16) || !aligned(codes, 16))
     return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -465,19 +465,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // with round-to-nearest-even and saturation to +-448.
 // ---------------------------------------------------------------------------
 template <typename TW>
-__global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const TW* __restrict__ w,
-                                                                int64_t rows, int cols,
-                                                                uint8_t* __restrict__ codes,
-                                                                float* __restrict__ scales,
-                                                                const int32_t* tiles_end = nullptr) {
-  // tiles_end (optional): rows beyond *tiles_end * 128 are left alone (the
-  // permuted buffers' unused tail)
-  if (tiles_end != nullptr) rows = min(rows, (int64_t)(*tiles_end) * ROW_TILE);
+__global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
+    const TW* __restrict__ w, int64_t rows, int cols, uint8_t* __restrict__ codes,
+    float* __restrict__ scales, const int32_t* __restrict__ tile_start = nullptr,
+    const int32_t* __restrict__ counts = nullptr, int E = 0, int64_t C = -1) {
+  // Rows of the permuted buffers (tile_start given): only the rows an expert
+  // actually holds (min(count, C) at the head of its 128-row segments) are
+  // quantised; the padding rows behind them are left alone.
+  if (tile_start != nullptr) rows = min(rows, (int64_t)tile_start[E] * ROW_TILE);
+  constexpr int VN = Vec16<TW>::N;  // elements per 16-byte vector
+  const int nvec = cols / VN;       // cols is a multiple of 16
   __shared__ float red[8];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const TW* wr = w + r * cols;
+    if (tile_start != nullptr) {
+      int lo = 0, hi = E - 1;  // the expert whose segment holds row r
+      const int tr = (int)(r / ROW_TILE);
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= tr) lo = mid; else hi = mid - 1;
+      }
+      const int64_t kept = C < 0 ? counts[lo] : min((int64_t)counts[lo], C);
+      if (r - (int64_t)tile_start[lo] * ROW_TILE >= kept) continue;  // block-uniform
+    }
+    const uint4* wr = reinterpret_cast<const uint4*>(w + r * cols);
     float m = 0.f;
-    for (int c = threadIdx.x; c < cols; c += blockDim.x) m = fmaxf(m, fabsf(to_f32(wr[c])));
+    for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+      float f[VN];
+      Vec16<TW>::unpack(ld_nc_v4(wr + c), f);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) m = fmaxf(m, fabsf(f[i]));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -486,8 +503,26 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const TW* __rest
 #pragma unroll
     for (int i = 0; i < 8; ++i) absmax = fmaxf(absmax, red[i]);
     const float scale = absmax > 0.f ? absmax / 448.0f : 1.0f;
-    for (int c = threadIdx.x; c < cols; c += blockDim.x)
-      codes[r * cols + c] = __nv_cvt_float_to_fp8(to_f32(wr[c]) / scale, __NV_SATFINITE, __NV_E4M3);
+    uint8_t* cr = codes + r * cols;
+    for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+      float f[VN];
+      Vec16<TW>::unpack(ld_nc_v4(wr + c), f);
+      uint32_t packed[VN / 4];
+#pragma unroll
+      for (int j = 0; j < VN / 4; ++j) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          v |= static_cast<uint32_t>(
+                   __nv_cvt_float_to_fp8(f[4 * j + i] / scale, __NV_SATFINITE, __NV_E4M3))
+               << (8 * i);
+        packed[j] = v;
+      }
+      if (VN == 8)
+        *reinterpret_cast<uint2*>(cr + c * VN) = make_uint2(packed[0], packed[VN / 4 - 1]);
+      else
+        *reinterpret_cast<uint32_t*>(cr + c * VN) = packed[0];
+    }
     if (threadIdx.x == 0) scales[r] = scale;
     __syncthreads();
   }
