@@ -16,7 +16,9 @@
 // multiply replaces the loop over experts).
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
-// MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// MMA issuer, warps 2..5 and 7..10 = epilogue (warp w reads TMEM lanes
+// 32*(w%4)..+31; the two warps of a quadrant split its column chunks), warp 6 =
+// second producer.
 // TMEM holds two 128x256 fp32 accumulators (512 columns), so the epilogue of
 // one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded: on expiry the kernel records
@@ -34,7 +36,11 @@ constexpr int BN = 256;            // accumulator columns per tile (UMMA N)
 constexpr int BK = 64;             // K per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;         // K of one tcgen05.mma kind::f16
 constexpr int B_BYTES = BN * BK * 2;
-constexpr int NUM_THREADS = 192;
+// warp 0 producer, 1 MMA, 2-5 epilogue (first half of the columns), 6 second
+// producer, 7-10 epilogue (second half)
+constexpr int NUM_THREADS = 352;
+constexpr int PROD2_WARP = 6;
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr int BAR_BYTES = 256;
@@ -352,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);  // one arrival per epilogue warp
+      mbar_init(tempty_bar(a), EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -376,21 +382,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const unsigned long long tmo = p.timeout_ns;
   const unsigned long long drain_tmo = p.drain_timeout_ns;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == PROD2_WARP) {
+    // ------------------------------------------------------------ producers
+    // Two producer threads take alternate K steps of the same walk (the step's
+    // stage is its running index modulo STAGES), so each thread's serial chain
+    // of wait, expect_tx and copies covers only every other stage.
     if (lane == 0) {
+      const uint32_t me = warp == 0 ? 0u : 1u;
       for (int g = 0; g < p.num_groups; ++g) {
         prefetch_map(&maps.a[g]);
         prefetch_map(&maps.b0[g]);
         if (EPI == EPI_SWIGLU_TC) prefetch_map(&maps.b1[g]);
       }
-      int stage = 0;
-      uint32_t phase = 0, issued = 0, last_par = 0;
+      uint32_t issued = 0, last_par = 0;
+      long long gs = 0;  // running K-step index over this CTA's tiles
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile(tile, tiles0, p, s_ts);
         const int kbs = p.g[ti.g].k_blocks;
-        for (int kb = 0; kb < kbs; ++kb) {
+        for (int kb = 0; kb < kbs; ++kb, ++gs) {
+          if ((uint32_t)(gs & 1) != me) continue;
+          const int stage = (int)(gs % STAGES);
+          const uint32_t phase = (uint32_t)((gs / STAGES) & 1);
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const uint32_t sa = stage0 + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
@@ -405,10 +418,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {  // let every copy already issued land before the CTA exits
+      if (!ok) {  // let every copy this thread issued land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
           if ((issued >> s) & 1u) wait_drain(full_bar(s), (last_par >> s) & 1u, drain_tmo);
       }
@@ -453,7 +465,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Two warps per TMEM lane quadrant, each taking every other 32-column chunk
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int half = warp >= 7 ? 1 : 0;
     const int r_in_tile = quad * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -475,7 +489,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float* bs1 = Q8 ? g.b_scale1 + (int64_t)ti.e * g.b_scale_stride : nullptr;
       if (EPI == EPI_SWIGLU_TC) {
 #pragma unroll 1
-        for (int c = 0; c < (BN / 2) / 32; ++c) {
+        for (int c = half; c < (BN / 2) / 32; c += 2) {
           float gv[32], uv[32];
           __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
           tmem_ld32(tb + c * 32, gv);
@@ -502,7 +516,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         const float sc = ((row_ok && g.row_scale != nullptr) ? g.row_scale[row] : 1.f) * ars;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           float v[32];
           __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the stores
           tmem_ld32(tb + c * 32, v);
