@@ -17,7 +17,7 @@
 //             (cp.async.bulk.tensor.cta_group::2 may signal the peer's barrier)
 //   empty[s]  both CTAs: the leader's tcgen05.commit multicast to both
 //   tfull[a]  both CTAs: the leader's commit multicast to both
-//   tempty[a] leader only: 4 epilogue warps of each CTA arrive (remote for the peer)
+//   tempty[a] leader only: 8 epilogue warps of each CTA arrive (remote for the peer)
 // Rows are grouped per expert in 128-row segments; a pair tile covers two
 // consecutive 128-row tiles of one expert, and when an expert has an odd tile
 // count the peer half of its last pair is computed but not stored.
@@ -37,7 +37,10 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = HALF_M * BK * 2;   // 16 KB
 constexpr int B_BYTES = 128 * BK * 2;      // 16 KB (this CTA's half of B)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+// warp 0 producer, 1 MMA, 2-5 and 6-9 epilogue (two warps per TMEM lane
+// quadrant, each taking every other 32-column chunk)
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES =
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(tfull_bar(a), 1);
-      tc::mbar_init(tempty_bar(a), 8);  // 4 epilogue warps in each of the two CTAs
+      tc::mbar_init(tempty_bar(a), 2 * EPI_WARPS);  // the epilogue warps of both CTAs
     }
     tc::mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -371,6 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quad = warp & 3;
+    const int half = warp >= 6 ? 1 : 0;
     const int r_in_half = quad * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
     for (long long tile = cluster_id; tile < total; tile += num_clusters) {
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.N;
       if (EPI == tc::EPI_SWIGLU_TC) {
 #pragma unroll 1
-        for (int c = 0; c < (BN / 2) / 32; ++c) {
+        for (int c = half; c < (BN / 2) / 32; c += 2) {
           float gv[32], uv[32];
           __syncwarp();
           tc::tmem_ld32(tb + c * 32, gv);
@@ -411,7 +415,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         const float sc = (row_ok && g.row_scale != nullptr) ? g.row_scale[row] : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           float v[32];
           __syncwarp();
           tc::tmem_ld32(tb + c * 32, v);
