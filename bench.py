@@ -33,6 +33,11 @@ METRIC = "MoE-layer tokens/s and active TFLOP/s vs B200 bf16 roofline, Mixtral s
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# (workload, weights) -> DRAM bytes / algorithmic bytes of the gate/up kernel, from one ncu
+# capture of that kernel as built (profiles/); absent = not captured for the current build.
+TRAFFIC_RATIO = {("mixtral", "dtype"): 539.386880 / 545.259520}
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -319,6 +324,12 @@ def run_ours(args, rank, world, local_rank):
     else:
         achieved, peak, unit, work = bytes_up / (k_up / 1e3) / 1e9, hbm_peak, "GB/s", bytes_up
         peak_note = f"hbm_gbs (of {peaks_src})"
+    # DRAM traffic of the dominant kernel: ncu's dram bytes over the algorithmic bytes on a
+    # small case of the same kernel and per-expert load, times this launch's algorithmic
+    # bytes (profiles/tc_grouped_gemm_mixtral_shape.md); None where no capture of the
+    # kernel as built stands
+    traffic_ratio = TRAFFIC_RATIO.get((args.workload, args.weights))
+    traffic = traffic_ratio * bytes_up if traffic_ratio is not None else None
     roofline_ms = max(flops_active / (tensor_peak * 1e12), (w_bytes + act_bytes) / (hbm_peak * 1e9)) * 1e3
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -332,7 +343,10 @@ def run_ours(args, rank, world, local_rank):
                        activations="e4m3 rows + fp32 row scales in the experts" if act_fp8
                        else w.dtype),
         "roofline": {"bound": up_bound, "kernel": KERNEL_NAMES[4], "achieved": achieved,
-                     "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": None,
+                     "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": ("ncu dram bytes / algorithmic bytes = %.3f on the "
+                                        "T=1024 E=2 case, times this launch's algorithmic "
+                                        "bytes" % traffic_ratio) if traffic is not None else None,
                      "algorithmic_per_launch": work, "peak_source": peak_note},
         "layer": {"active_tflops": flops_active / (ms_step / 1e3) / 1e12,
                   "active_flops_per_step": flops_active, "touched_weight_bytes": w_bytes,

@@ -70,10 +70,11 @@ MIXTRAL_DECODE = Workload("mixtral-decode T=32 d=4096 E=8 d_e=14336 k=2", 32, 40
 
 ALL_WORKLOADS = (TINY_F32, MIXTRAL, DEEPSEEK_V3, SWITCH_ZIPF, MIXTRAL_DECODE)
 
-# A smaller case with the Mixtral expert shape (about 1 GB on the device), for
-# hardware-counter captures of the same kernels.
-MIXTRAL_PROFILE = Workload("mixtral-shape-profile T=2048 d=4096 E=2 d_e=14336 k=2",
-                           2048, 4096, 2, 14336, 2, seed=1)
+# A smaller case with the Mixtral expert shape and the full layer's load of
+# 1024 routed rows per expert (so the same kernel choices: 1-CTA gate/up, CTA
+# pairs for down), about 0.8 GB on the device, for hardware-counter captures.
+MIXTRAL_PROFILE = Workload("mixtral-shape-profile T=1024 d=4096 E=2 d_e=14336 k=2",
+                           1024, 4096, 2, 14336, 2, seed=1)
 # The decode shape with 2 experts (about 0.7 GB of bf16 weights), likewise.
 DECODE_PROFILE = Workload("decode-shape-profile T=32 d=4096 E=2 d_e=14336 k=2",
                           32, 4096, 2, 14336, 2, seed=4)
