@@ -146,7 +146,9 @@ typedef struct {
   void* stream;              /* cudaStream_t to enqueue on; NULL = default stream */
   void* const* events;       /* optional cudaEvent_t[2*MOE_NUM_KERNELS]; when non-NULL,
                                 events[2i] / events[2i+1] are recorded on `stream`
-                                right before / after kernel i (NULL entries skipped) */
+                                right before / after step i (NULL entries skipped);
+                                with MOE_WEIGHTS_FP8_W8A8 the x quantiser falls in the
+                                scatter step and the H quantiser in the down step */
   const float* selection_bias; /* device [E] fp32 added to the selection scores only
                                   (who is picked, not the gates), or NULL */
   int32_t n_group;           /* group-limited selection: experts form n_group contiguous
@@ -181,7 +183,7 @@ MOE_API int64_t moe_capacity(int64_t T, int E, int k, float capacity_factor);
  *   x        device [T, d]            dtype
  *   W_r      device [E, d]            fp32 (the router's d x E matrix, stored expert-major)
  *   W_g, W_u device [E, d_e, d]       dtype (nn.Linear weight layout: K contiguous),
- *                                    or uint8 E4M3 codes with MOE_WEIGHTS_FP8
+ *                                    or uint8 E4M3 codes with MOE_WEIGHTS_FP8(_W8A8)
  *   W_d      device [E, d, d_e]       dtype (or uint8 codes)
  *   W_shared device, packed [gate (d_s x d) | up (d_s x d) | down (d x d_s)], or
  *            NULL when dims->d_s == 0
@@ -189,7 +191,8 @@ MOE_API int64_t moe_capacity(int64_t T, int E, int k, float capacity_factor);
  *   aux      device float[1]          written: E * sum_i f_i P_i (0 when T == 0)
  *   counts   device int32[E]          written: routed assignments per expert,
  *                                     before the capacity cut
- * Enqueues MOE_NUM_KERNELS kernels on dims->stream, no host synchronisation.
+ * Enqueues MOE_NUM_KERNELS kernels on dims->stream (two more, the x and H
+ * quantisers, with MOE_WEIGHTS_FP8_W8A8), no host synchronisation.
  */
 MOE_API moe_status moe_forward(const moe_dims* dims,
                        const void* x, const float* W_r, const void* W_g,

@@ -1,6 +1,6 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (sm_100a):
 // TMA (cp.async.bulk.tensor, 128-byte swizzle) -> shared-memory ring ->
-// single-thread tcgen05.mma (bf16 x bf16 -> fp32 in TMEM) -> tcgen05.ld
+// single-thread tcgen05.mma (bf16 x bf16, or E4M3 x E4M3, -> fp32 in TMEM) -> tcgen05.ld
 // epilogue. Persistent: one CTA per SM walks a static tile list that it
 // derives on the device from the per-expert segment starts, so no host
 // synchronisation sits between routing and the expert products.
@@ -15,10 +15,12 @@
 // FFN_i(x) = (SiLU(x W_g) * x W_u) W_d) and "In PyTorch" (a grouped matrix
 // multiply replaces the loop over experts).
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
-// MMA issuer, warps 2..5 and 7..10 = epilogue (warp w reads TMEM lanes
-// 32*(w%4)..+31; the two warps of a quadrant split its column chunks), warp 6 =
-// second producer.
+// Warp roles (352 threads): warps 0 and 6 = TMA producers (alternate K steps),
+// warp 1 = TMEM owner and MMA issuer, warps 2..5 and 7..10 = epilogue (warp w
+// reads TMEM lanes 32*(w%4)..+31; the two warps of a quadrant split its column
+// chunks).
+// With Q8 (E4M3 operands, tcgen05 kind::f8f6f4) the same pipeline runs on code
+// tiles, 128 codes per K step, and the epilogue applies the operands' row scales.
 // TMEM holds two 128x256 fp32 accumulators (512 columns), so the epilogue of
 // one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded: on expiry the kernel records
