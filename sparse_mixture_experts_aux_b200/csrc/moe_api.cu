@@ -104,7 +104,7 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
   p.router_narrow = E <= 16;
   p.router_split = p.router_narrow ? moe::narrow_split_k(p.T, E, p.d)
-                                   : moe::simt_split_k(p.T, E, p.d);
+                                   : moe::router_wide_split_k(p.T, E, p.d);
   p.o_logits = take(static_cast<size_t>(p.router_split) * T * E * 4);
   p.o_idx = take(TK * 4);
   p.o_gate = take(TK * 4);
@@ -359,20 +359,6 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   const int T = static_cast<int>(P.T);
 
   // (0) router logits, fp32 FMA
-  moe::SimtGroup rg{};
-  rg.A = x;
-  rg.B0 = W_r;
-  rg.B1 = nullptr;
-  rg.b_stride = 0;
-  rg.C = logits;
-  rg.tile_start = nullptr;
-  rg.E = 1;
-  rg.rows = P.T;
-  rg.N = P.E;
-  rg.K = P.d;
-  rg.active = 1;
-  rg.split_k = P.router_split;
-  moe::SimtGroup none{};
   tm.at(0);
   if (P.router_narrow) {
     if (P.E <= 8) {
@@ -385,9 +371,10 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
           <<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split, logits);
     }
   } else {
-    dim3 grid((P.E + moe::SG_BN - 1) / moe::SG_BN, (T + moe::SG_BM - 1) / moe::SG_BM,
+    dim3 grid((P.E + moe::RW_BN - 1) / moe::RW_BN, (T + moe::RW_BM - 1) / moe::RW_BM,
               P.router_split);
-    moe::simt_gemm_kernel<TX, float, float, moe::EPI_STORE_F32><<<grid, 256, 0, st>>>(rg, none);
+    moe::router_wide_kernel<TX><<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split,
+                                                       logits);
   }
   tm.at(1);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;

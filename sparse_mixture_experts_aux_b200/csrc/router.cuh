@@ -202,6 +202,104 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
 }
 
 // ---------------------------------------------------------------------------
+// Router logits for many experts (E > 16): r[t, e] = sum_j x[t, j] W_r[e, j]
+// in fp32 FMA. 128 tokens x 128 experts per block, 256 threads, each thread
+// 8 tokens x 8 experts, so a K step reads 16 operand values from shared memory
+// for 64 FMAs. The sum is blocked like the generic kernel's: 32-term partials
+// added to the accumulator, in a fixed order; grid.z splits K into
+// RW_BK-multiple ranges whose partials the routing kernel adds in order.
+// ---------------------------------------------------------------------------
+constexpr int RW_BM = 128, RW_BN = 128, RW_BK = 32;
+
+// K splits for the wide router: enough blocks to fill the SMs; K ranges stay
+// whole multiples of RW_BK. Depends only on the shape.
+inline int router_wide_split_k(int64_t T, int E, int K) {
+  const int64_t blocks = ((E + RW_BN - 1) / RW_BN) * ((T + RW_BM - 1) / RW_BM);
+  int split = 1;
+  while (blocks * split < 296 && (K % (2 * split * RW_BK)) == 0 && K / (2 * split) >= 512)
+    split *= 2;
+  return split;
+}
+
+template <typename TA>
+__global__ void __launch_bounds__(256, 1) router_wide_kernel(const TA* __restrict__ x,
+                                                             const float* __restrict__ W_r,
+                                                             int T, int K, int E, int splits,
+                                                             float* __restrict__ logits) {
+  __shared__ __align__(16) float As[RW_BK][RW_BM + 4];
+  __shared__ __align__(16) float Bs[RW_BK][RW_BN + 4];
+  const int k_len = K / splits;
+  const int k_begin = (int)blockIdx.z * k_len;
+  const int n0 = blockIdx.x * RW_BN;
+  const int m0 = blockIdx.y * RW_BM;
+  const int tid = threadIdx.x;
+  const int lr = tid >> 1, lk = (tid & 1) * 16;  // staging: row lr, K elements lk .. lk+15
+  const int ty = tid >> 4, tx = tid & 15;         // compute: rows 8ty.., columns 8tx..
+  const bool a_ok = m0 + lr < T, b_ok = n0 + lr < E;
+  const TA* arow = x + (int64_t)(m0 + lr) * K;
+  const float* brow = W_r + (int64_t)(n0 + lr) * K;
+  float fa[16], fb[16];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (a_ok) load4<TA>(arow + k0 + lk + 4 * q, fa + 4 * q);
+      else fa[4 * q] = fa[4 * q + 1] = fa[4 * q + 2] = fa[4 * q + 3] = 0.f;
+      if (b_ok) load4<float>(brow + k0 + lk + 4 * q, fb + 4 * q);
+      else fb[4 * q] = fb[4 * q + 1] = fb[4 * q + 2] = fb[4 * q + 3] = 0.f;
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  fetch(k_begin);
+  for (int k0 = k_begin; k0 < k_begin + k_len; k0 += RW_BK) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      As[lk + i][lr] = fa[i];
+      Bs[lk + i][lr] = fb[i];
+    }
+    __syncthreads();
+    if (k0 + RW_BK < k_begin + k_len) fetch(k0 + RW_BK);  // in flight during the compute
+    float part[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) part[i][j] = 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < RW_BK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] += part[i][j];
+    __syncthreads();
+  }
+  float* C = logits + (int64_t)blockIdx.z * T * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + ty * 8 + i;
+    if (m >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + tx * 8 + j;
+      if (n < E) C[(int64_t)m * E + n] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Router logits for few experts (E <= NE, NE = 8 or 16): r[t, e] = sum_j x[t, j] W_r[e, j].
 // This is bound by reading x, so there is no wasted output tile. A block
 // owns NARROW_TB tokens and one K range (grid.y splits K; the routing kernel
