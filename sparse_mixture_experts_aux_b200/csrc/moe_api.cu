@@ -717,8 +717,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   {
     moe::SimtGroup a{}, b{};
     a = {xp, W_g, W_u, static_cast<int64_t>(P.de) * P.d, h, nullptr, tile_start, E, 0, P.de, P.d,
-         1, 1};
-    if (P.ds) b = {xf, sg, sg + sh_n, 0, hs, nullptr, nullptr, 1, P.T, P.ds, P.d, 1, 1};
+         1};
+    if (P.ds) b = {xf, sg, sg + sh_n, 0, hs, nullptr, nullptr, 1, P.T, P.ds, P.d, 1};
     const int nmax = P.de > P.ds ? P.de : P.ds;
     dim3 grid((nmax + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
@@ -730,8 +730,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   {
     moe::SimtGroup a{}, b{};
     a = {h, W_d, nullptr, static_cast<int64_t>(P.d) * P.de, yrows, rowgate, tile_start, E, 0, P.d,
-         P.de, 1, 1};
-    if (P.ds) b = {hs, sg + 2 * sh_n, nullptr, 0, ys, nullptr, nullptr, 1, P.T, P.d, P.ds, 1, 1};
+         P.de, 1};
+    if (P.ds) b = {hs, sg + 2 * sh_n, nullptr, 0, ys, nullptr, nullptr, 1, P.T, P.d, P.ds, 1};
     dim3 grid((P.d + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
     tm.at(10);

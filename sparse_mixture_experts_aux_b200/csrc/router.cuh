@@ -16,39 +16,27 @@ namespace moe {
 
 // ---------------------------------------------------------------------------
 // SIMT fp32 "TN" GEMM: C[m, n] = sum_k A[m, k] * B[e][n, k], both operands
-// K-contiguous, fp32 FMA accumulation (no TF32). Used for the router logits
-// (A = x, B = W_r) and for the fp32 layer's expert products, where the
-// rows of A are grouped per expert in ROW_TILE-padded segments.
+// K-contiguous, fp32 FMA accumulation (no TF32). Used for the fp32 layer's
+// expert products, where the rows of A are grouped per expert in
+// ROW_TILE-padded segments; grid z selects the routed or the shared group.
 // ---------------------------------------------------------------------------
-enum { EPI_STORE_F32 = 0, EPI_SWIGLU = 1, EPI_SCALE = 2 };
+enum { EPI_SWIGLU = 1, EPI_SCALE = 2 };
 
 struct SimtGroup {
   const void* A;            // [rows, K]
   const void* B0;           // expert e at B0 + e * b_stride  ([N, K] each)
   const void* B1;           // second operand of the SwiGLU (up projection)
   int64_t b_stride;         // elements between experts
-  void* C;                  // [rows, N]; with split_k > 1: [split_k][rows][N] partial sums
+  void* C;                  // [rows, N]
   const float* row_scale;   // EPI_SCALE: multiplier per row (NULL = 1)
   const int32_t* tile_start;// grouped rows: [E + 1] segment starts in ROW_TILE units; NULL = dense
   int E;
   int64_t rows;             // dense: number of valid rows
   int N, K;
   int active;               // 0: this grid z-slice does nothing
-  int split_k;              // > 1 (EPI_STORE_F32 only): grid z splits K into equal chunks
 };
 
 constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 32;
-
-// Number of K chunks for a dense fp32-output product of rows x N x K: enough
-// blocks to fill the GPU several times over, chunks of at least 256 and a
-// multiple of SG_BK. Depends only on the shape, so the workspace size does too.
-inline int simt_split_k(int64_t rows, int N, int K) {
-  const int64_t blocks = ((N + SG_BN - 1) / SG_BN) * ((rows + SG_BM - 1) / SG_BM);
-  int split = 1;
-  while (blocks * split < 600 && (K % (2 * split * SG_BK)) == 0 && K / (2 * split) >= 256)
-    split *= 2;
-  return split;
-}
 
 template <typename TA>
 __device__ __forceinline__ void load4(const TA* p, float* f);
@@ -72,12 +60,10 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
 // the rounding error of a long dot product well below one sequential chain.
 template <typename TA, typename TB, typename TC, int EPI>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup g1) {
-  const bool splitting = g0.split_k > 1;
-  const SimtGroup g = (splitting || blockIdx.z == 0) ? g0 : g1;
+  const SimtGroup g = blockIdx.z == 0 ? g0 : g1;
   if (!g.active) return;
-  const int split = splitting ? (int)blockIdx.z : 0;
-  const int k_len = splitting ? g.K / g.split_k : g.K;
-  const int k_begin = split * k_len;
+  const int k_len = g.K;
+  const int k_begin = 0;
   const int n0 = blockIdx.x * SG_BN;
   const int64_t m0 = (int64_t)blockIdx.y * SG_BM;
   if (n0 >= g.N) return;
@@ -176,7 +162,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup 
     __syncthreads();
   }
 
-  TC* C = reinterpret_cast<TC*>(g.C) + (splitting ? (int64_t)split * g.rows * g.N : 0);
+  TC* C = reinterpret_cast<TC*>(g.C);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t m = m0 + ty * 4 + i;
