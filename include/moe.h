@@ -57,7 +57,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, NaN factor */
-  MOE_ERR_UNSUPPORTED = 2,    /* valid layer this build does not run (see limits below) */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid layer this library does not run (see limits below) */
   MOE_ERR_WORKSPACE = 3,      /* workspace null, too small or misaligned */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
   MOE_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up (moe_get_device_status) */
@@ -73,7 +73,7 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * + gate scaling, combine (un-permute + shared expert). */
 #define MOE_NUM_KERNELS 7
 
-/* Limits of this build: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
+/* Limits of this library: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
  * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1);
  * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group. */
 
