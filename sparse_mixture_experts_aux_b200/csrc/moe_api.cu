@@ -829,8 +829,22 @@ moe_status moe_forward_host_io(const moe_dims* dims, const void* x_host, void* x
       cudaMemcpyAsync(counts_host, counts_dev, sizeof(int32_t) * E, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
-  return moe_get_device_status();
+  // the status word is read in order on this stream (a synchronous symbol copy
+  // would wait on the legacy default stream and so on other callers' work)
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, moe::g_dev_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(moe::g_dev_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
 }
 
 const char* moe_status_string(moe_status s) {
