@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= CONV_WARP0 && warp < CONV_WARP0 + CONV_WARPS) {
     // ---------------------------------------------------------------- converters
     // For chunk g, 256 threads turn half (g & 1) of the Q tile (chunks 4h..4h+3
-    // of each 128-byte row, stored at chunk ^ (row & 7)) into the bf16 tile: 16
+    // of each 128-byte row, stored at chunk ^ (row & 7)) into the fp16 tile: 16
     // codes -> two 16-byte chunks at (2c, 2c+1) ^ (row & 7). A thread owns rows
     // r, r+64, r+128, r+192 with r & 7 = its lane & 7, so the 8 lanes of every
     // shared-memory phase hit 8 different 16-byte bank groups, both when reading
