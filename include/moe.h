@@ -75,7 +75,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
 /* Limits of this library: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
  * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1);
- * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group. */
+ * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group; the FP8
+ * weight formats need bf16 x and no shared expert (d_s = 0). */
 
 /*
  * Routing variants (gate_mode, selection_bias, n_group / topk_group).
@@ -123,8 +124,9 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * FP8 on both GEMM operands (W8A8): the weights as for MOE_WEIGHTS_FP8, and
  * the routed experts' inputs quantised the same way, one fp32 scale per row:
  * each token row of x (absmax over d) and each routed hidden row H (absmax
- * over d_e) becomes E4M3 codes * scale. The expert GEMMs then run E4M3 x E4M3
- * -> fp32 on the tensor cores, and both scales multiply the accumulator. This
+ * over d_e, after H is rounded to bf16) becomes E4M3 codes * scale. The expert
+ * GEMMs then run E4M3 x E4M3 -> fp32 on the tensor cores, and both scales
+ * multiply the accumulator. This
  * changes the numbers (activations carry 3 mantissa bits): it is a different
  * layer from MOE_WEIGHTS_FP8, not a faster route to the same one.
  */
