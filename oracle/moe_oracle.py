@@ -55,6 +55,8 @@ __all__ = [
     "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
     "E4M3_MAX", "e4m3_round", "e4m3_encode", "e4m3_decode", "quantize_rows_fp8",
     "dequantize_rows_fp8", "fake_quant_rows_fp8", "round_bf16", "swiglu_ffn_w8a8",
+    "E2M1_MAX", "MX_BLOCK", "e2m1_round", "e2m1_encode", "e2m1_decode", "quantize_rows_mxfp4",
+    "dequantize_rows_mxfp4",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
     "moe_param_count", "active_flops", "OracleResult",
 ]
@@ -436,6 +438,73 @@ def quantize_rows_fp8(w):
 def dequantize_rows_fp8(codes, scales) -> np.ndarray:
     """The weights the layer computes with: code value times the row scale (fp64, exact)."""
     return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
+
+
+# R14 (MXFP4, the 4-bit format the pages name for gpt-oss's expert weights;
+# AI Engineering Illustrated "Mixture of Experts", "Trade-offs to weigh"): the
+# pages give no format details, so the reading follows the Open Compute
+# microscaling convention: blocks of 32 consecutive weights along K share one
+# power-of-two scale X = 2^(floor(log2(absmax)) - 2) (2 = the largest E2M1
+# exponent; X = 1 for an all-zero block), and each weight becomes the E2M1
+# value nearest to w / X (1 sign, 2 exponent bits with bias 1, 1 mantissa bit:
+# magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even mantissa, saturated
+# at +-6. The layer would compute with code_value * X.
+E2M1_MAX = 6.0
+MX_BLOCK = 32
+
+
+def e2m1_round(v) -> np.ndarray:
+    """Nearest E2M1 value (ties to even), saturated to +-6, as float64. The
+    spacing is 0.5 below 2, 1 in [2, 4) and 2 from 4 on."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    q = np.where(a < 2.0, 0.5, np.where(a < 4.0, 1.0, 2.0))
+    r = np.minimum(np.rint(a / q) * q, E2M1_MAX)
+    return np.copysign(r, v)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """4-bit codes (sign << 3 | exponent << 1 | mantissa), one per uint8."""
+    r = e2m1_round(v)
+    a = np.abs(r)
+    sign = np.signbit(r).astype(np.uint8) << 3
+    normal = a >= 1.0
+    e = np.floor(np.log2(np.where(normal, a, 1.0))).astype(np.int64)
+    mant_n = np.rint(a / 2.0 ** e * 2 - 2).astype(np.int64)
+    code = np.where(normal, ((e + 1) << 1) | mant_n, np.rint(a / 0.5).astype(np.int64))
+    return (sign | code.astype(np.uint8)).astype(np.uint8)
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """float64 values of 4-bit E2M1 codes."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    val = np.where(e == 0, m * 0.5, (1.0 + m / 2.0) * 2.0 ** (e - 1))
+    return s * val
+
+
+def quantize_rows_mxfp4(w):
+    """Per-block MXFP4 quantisation (R14) of a [rows, K] matrix, K a multiple of
+    32; returns (codes uint8 [rows, K], one code per element, and the blocks'
+    scale exponents int64 [rows, K / 32], X = 2^exponent)."""
+    w32 = np.asarray(_f64(w), dtype=np.float32)
+    rows, K = w32.shape
+    blocks = w32.reshape(rows, K // MX_BLOCK, MX_BLOCK).astype(np.float64)
+    amax = np.abs(blocks).max(axis=2)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))  # amax = f * 2^ex, f in [0.5, 1)
+    exps = np.where(amax > 0, (ex - 1) - 2, 0).astype(np.int64)
+    codes = e2m1_encode(blocks / np.ldexp(1.0, exps)[:, :, None])
+    return codes.reshape(rows, K), exps
+
+
+def dequantize_rows_mxfp4(codes, exps) -> np.ndarray:
+    """code value * 2^exponent of its block (fp64, exact)."""
+    c = np.asarray(codes)
+    rows, K = c.shape
+    vals = e2m1_decode(c).reshape(rows, K // MX_BLOCK, MX_BLOCK)
+    return (vals * np.ldexp(1.0, np.asarray(exps))[:, :, None]).reshape(rows, K)
 
 
 # R13 (FP8 on both operands): the GEMM inputs of a routed expert, the token
