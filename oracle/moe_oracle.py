@@ -529,13 +529,12 @@ def swiglu_ffn_w8a8(x, W_g, W_u, W_d) -> np.ndarray:
     """One SwiGLU expert with E4M3 activations (R13): x rows quantised per row,
     the gate/up GEMM, SwiGLU in full precision, H rows quantised per row, the
     down GEMM. W_g, W_u, W_d are the weights the layer computes with (for FP8
-    weights: code * scale). R13b: H is held in bf16 before its quantisation (the
-    precision the layer stores it in), so that both sides decide H's codes from
-    the same values."""
+    weights: code * scale). H is quantised from its fp64 value: the pages fix
+    no storage precision for it, and every step after the router is fp64 (R2)."""
     xq = fake_quant_rows_fp8(_f64(x))
     a = xq @ _f64(W_g).T
     b = xq @ _f64(W_u).T
-    hq = fake_quant_rows_fp8(round_bf16(silu(a) * b))
+    hq = fake_quant_rows_fp8(silu(a) * b)
     return hq @ _f64(W_d).T
 
 

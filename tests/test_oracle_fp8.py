@@ -91,7 +91,6 @@ def test_w8a8_ffn_against_library_assembled_reference():
     xq = _torch_fake_quant_rows(x)
     a, b = xq @ Wg.T, xq @ Wu.T
     h = (a / (1.0 + np.exp(-a))) * b
-    h = torch.tensor(h, dtype=torch.float32).to(torch.bfloat16).double().numpy()
     ref = _torch_fake_quant_rows(h) @ Wd.T
     got = O.swiglu_ffn_w8a8(x, Wg, Wu, Wd)
     assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
@@ -111,11 +110,10 @@ def test_w8a8_ffn_is_exact_on_representable_inputs():
     Wg = np.zeros((1, 64)); Wg[0, 1] = 1.0
     Wu = np.zeros((1, 64)); Wu[0, 0] = 1.0 / 448.0
     Wd = np.ones((1, 1))
-    h = O.round_bf16(O.silu(x[:, 1]) * 1.0)
+    h = O.silu(x[:, 1]) * 1.0
     got = O.swiglu_ffn_w8a8(x, Wg, Wu, Wd)[:, 0]
-    # a single-entry row quantises to +-448 * (|h| / 448): the bf16 value of h
-    # up to the fp32 rounding of its scale
-    assert np.allclose(got, h, rtol=2.0 ** -22)
+    # a single-entry row quantises to +-448 * (|h| / 448) exactly up to fp32 rounding of h
+    assert np.allclose(got, h, rtol=2.0 ** -23)
 
 
 def test_round_bf16_is_rne_through_fp32():
