@@ -319,3 +319,86 @@ def test_aux_top1_variant_agrees_at_k1():
 def test_dropped_fraction_from_counts():
     assert O.dropped_fraction(np.array([3000, 2000, 1500, 1692]), 2560, 4096, 2) == pytest.approx(440 / 8192)
     assert O.dropped_fraction(np.array([5, 5]), None, 5, 2) == 0.0
+
+
+# --- the routing margin that decides which tokens parity compares ----------
+
+def _separation_brute(row, k):
+    """The largest gap by which some k-subset of `row` sits above the rest:
+    max over k-subsets S of (min over S) - (max outside S). The top-k set
+    attains it, so it is the k-th/(k+1)-th gap, found without sorting."""
+    n = len(row)
+    if k >= n:
+        return math.inf
+    best = -math.inf
+    for S in itertools.combinations(range(n), k):
+        inside = min(row[i] for i in S)
+        outside = max(row[j] for j in range(n) if j not in S)
+        best = max(best, inside - outside)
+    return best
+
+
+def test_topk_margin_brute_force_tiny():
+    rng = np.random.default_rng(40)
+    for E in (2, 3, 5, 7):
+        r = rng.normal(size=(25, E))
+        r[:5] = np.round(r[:5], 1)  # repeated values, ties at the cut included
+        for k in range(1, E + 1):
+            got = O.topk_margin(r, k)
+            want = np.array([_separation_brute(list(row), k) for row in r])
+            assert np.array_equal(got, want), (E, k)
+
+
+def test_topk_margin_hand_cases():
+    r = np.array([[5.0, 4.0, 2.0, 1.0],    # k=2: 4 - 2, not 2 - 1 nor 5 - 4
+                  [1.0, 3.0, 3.0, 0.0],    # k=1: a tie at the cut gives 0
+                  [0.5, 0.5, 0.5, 0.5]])
+    assert O.topk_margin(r, 2).tolist() == [2.0, 2.0, 0.0]
+    assert O.topk_margin(r, 1).tolist() == [1.0, 0.0, 0.0]
+    assert np.isinf(O.topk_margin(r, 4)).all()
+
+
+def test_group_gap_and_selection_gap_brute_force():
+    # group scores and the kept groups by hand; both gaps by the subset brute force
+    rng = np.random.default_rng(41)
+    E, n_group, topk_group, k = 12, 4, 2, 3
+    gsize = E // n_group
+    sel = rng.normal(size=(50, E))
+    sel[:6] = np.round(sel[:6], 1)
+    el, gap = O.group_eligible(sel, n_group, topk_group)
+    idx, kgap = O.select_experts(sel, k, el)
+    for t in range(50):
+        gbest = [max(sel[t, g * gsize:(g + 1) * gsize]) for g in range(n_group)]
+        assert gap[t] == _separation_brute(gbest, topk_group)
+        groups = sorted(range(n_group), key=lambda g: (-gbest[g], g))[:topk_group]
+        allowed = [e for e in range(E) if e // gsize in groups]
+        assert el[t].tolist() == [e in allowed for e in range(E)]
+        assert kgap[t] == _separation_brute([sel[t, e] for e in allowed], k)
+    # every group kept, or one pick per allowed expert: no gap can matter
+    assert np.isinf(O.group_eligible(sel, n_group, n_group)[1]).all()
+    _, kg = O.select_experts(sel, topk_group * gsize, el)
+    assert np.isinf(kg).all()
+
+
+def test_layer_margin_is_the_smaller_gap_on_the_selection_scores():
+    # the layer's margin is taken on what the top-k ranks (affinity + selection
+    # bias in sigmoid mode), and is the smaller of the group and the expert gap
+    rng = np.random.default_rng(42)
+    T, d, E, k, ng, tg = 30, 8, 8, 2, 4, 2
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(E, d))
+    b = rng.normal(scale=0.05, size=E)
+    res = O.moe_forward(x, Wr, lambda e: None, k, rows=np.array([], dtype=int),
+                        gate_mode=O.GATE_SIGMOID, selection_bias=b, n_group=ng, topk_group=tg)
+    gsize = E // ng
+    for t in range(T):
+        s = [1.0 / (1.0 + math.exp(-res.logits[t, e])) + b[e] for e in range(E)]
+        gbest = [max(s[g * gsize:(g + 1) * gsize]) for g in range(ng)]
+        groups = sorted(range(ng), key=lambda g: (-gbest[g], g))[:tg]
+        allowed = [s[e] for e in range(E) if e // gsize in groups]
+        want = min(_separation_brute(gbest, tg), _separation_brute(allowed, k))
+        assert res.margin[t] == pytest.approx(want, rel=1e-12, abs=1e-15)
+    # with plain renormalised routing it is the logit gap
+    res0 = O.moe_forward(x, Wr, lambda e: None, k, rows=np.array([], dtype=int))
+    want0 = [_separation_brute(list(res0.logits[t]), k) for t in range(T)]
+    assert res0.margin.tolist() == want0
