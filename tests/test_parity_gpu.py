@@ -69,7 +69,9 @@ def test_mixtral_workload_sampled():
 
 def test_switch_zipf_workload_sampled():
     r = check_workload(SWITCH_ZIPF, sample=256)
-    assert r["excluded"] <= SWITCH_ZIPF.T
+    print(f"switch: {r['rows_compared']} of {r['rows_sampled']} sampled rows compared, "
+          f"{r['near_ties']} near-tie tokens, {r['excluded']} tokens excluded")
+    assert r["rows_compared"] >= 200
 
 
 def test_deepseek_v3_workload_sampled():

@@ -112,7 +112,7 @@ def test_w8a8_mixtral_sampled_rows():
     fp8 = make_fp8_weights(w, device="cuda")
     gpu = run_gpu(w, inp, fp8=fp8, act_fp8=True)
     inp.pop("W_g"), inp.pop("W_u"), inp.pop("W_d")
-    rows = np.sort(np.random.default_rng(5).choice(w.T, size=64, replace=False))
+    rows = np.sort(np.random.default_rng(5).choice(w.T, size=256, replace=False))
     compare(w, gpu, run_oracle(w, inp, rows=rows, fp8=fp8, act_fp8=True))
 
 
