@@ -8,10 +8,15 @@ One step = one moe_forward call over one batch of T tokens: router logits,
 routing, scan, scatter, gate/up GEMM + SwiGLU, down GEMM + gate scaling,
 combine. Weights and a ring of fresh x batches are resident in HBM before the
 timed region; the expert weights (2.8 GB for the Mixtral-shaped layer) are
-larger than L2, so no L2 flush is needed between steps. Under torchrun every
-rank runs its own replica on its own GPU ("replicas only": the layer has no
-exchange step); the job value is the tokens of all ranks over the slowest
-rank's device time. Rank 0 prints one JSON line.
+larger than L2, so no L2 flush is needed between steps. Every rank runs its
+own replica on its own GPU ("replicas only": the layer has no exchange step);
+the job value is the tokens of all ranks over the slowest rank's device time.
+Ranks come from torchrun's environment, or, when none is set and --gpus N > 1,
+from N processes this script spawns itself. Rank 0 prints one JSON line.
+
+The default (Mixtral-shaped) run also times the weight-streaming decode shape
+on the same weights: T = 32 tokens, 1000 back-to-back calls, each on its own
+pre-generated x, reported under "decode" against the HBM bandwidth.
 """
 from __future__ import annotations
 
@@ -38,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC_RATIO = {("mixtral", "dtype"): 539.386880 / 545.259520}
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
@@ -46,21 +51,25 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral",
                     choices=["mixtral", "deepseek_v3", "switch_zipf", "decode", "tiny_fp32",
-                             "mixtral_profile", "decode_profile"])
+                             "mixtral_profile", "decode_profile", "routing_profile"])
     ap.add_argument("--weights", choices=["dtype", "fp8", "w8a8"], default="dtype",
                     help="expert weights in the activation dtype; E4M3 codes with per-row "
                          "scales (quantised once by the library before timing); or those and "
                          "E4M3 activations inside the experts (W8A8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode-shape leg of the default Mixtral-shaped run")
+    ap.add_argument("--decode-calls", type=int, default=1000)
+    return ap.parse_args(argv)
 
 
 def workload_by_name(name):
     from sparse_mixture_experts_aux_b200 import inputs as I
     return {"mixtral": I.MIXTRAL, "deepseek_v3": I.DEEPSEEK_V3, "switch_zipf": I.SWITCH_ZIPF,
             "decode": I.MIXTRAL_DECODE, "tiny_fp32": I.TINY_F32,
-            "mixtral_profile": I.MIXTRAL_PROFILE, "decode_profile": I.DECODE_PROFILE}[name]
+            "mixtral_profile": I.MIXTRAL_PROFILE, "decode_profile": I.DECODE_PROFILE,
+            "routing_profile": I.ROUTING_PROFILE}[name]
 
 
 def load_peaks():
@@ -214,6 +223,64 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------------------- our arm
+def step_work(w, counts, fp8: bool):
+    """Algorithmic work of one step from its own routing counts: kept
+    assignments, touched experts, FLOPs of the two GEMMs, and the bytes each
+    GEMM and the whole layer must move at least (touched expert weights once,
+    plus the rows a GEMM reads and writes; x in and y out for the layer)."""
+    from sparse_mixture_experts_aux_b200 import _lib
+    C = _lib.moe_capacity(w.T, w.E, w.k, w.capacity_factor)
+    C = None if C < 0 else C
+    kept_e = [int(c) if C is None else min(int(c), C) for c in counts]
+    kept = sum(kept_e)
+    touched = sum(1 for c in kept_e if c > 0)
+    esz = 2 if w.dtype == "bf16" else 4
+    wsz = 1 if fp8 else esz  # bytes per expert weight (+ 4 per row of scales with FP8)
+    sh = w.T if w.d_s else 0
+    flops_up = 2 * kept * w.d * 2 * w.d_e + 2 * sh * w.d * 2 * w.d_s
+    flops_down = 2 * kept * w.d_e * w.d + 2 * sh * w.d_s * w.d
+    bytes_up = (touched * 2 * w.d * w.d_e * wsz + (touched * 2 * w.d_e * 4 if fp8 else 0)
+                + 2 * w.d * w.d_s * esz + (kept * (w.d + w.d_e) + sh * (w.d + w.d_s)) * esz)
+    bytes_down = (touched * w.d * w.d_e * wsz + (touched * w.d * 4 if fp8 else 0)
+                  + w.d * w.d_s * esz + (kept * (w.d_e + w.d) + sh * (w.d_s + w.d)) * esz)
+    w_bytes = (touched * 3 * w.d * w.d_e * wsz + (touched * 2 * (w.d_e + w.d) * 4 if fp8 else 0)
+               + 3 * w.d * w.d_s * esz + w.E * w.d * 4)
+    return dict(C=C, kept=kept, touched=touched, flops_up=flops_up, flops_down=flops_down,
+                flops=flops_up + flops_down, bytes_up=bytes_up, bytes_down=bytes_down,
+                w_bytes=w_bytes, act_bytes=2 * w.T * w.d * esz)
+
+
+def kernel_roofline(flops, nbytes, ms, tensor_peak, hbm_peak):
+    """The kernel's bound (the slower of its FLOPs at tensor peak and its
+    algorithmic bytes at HBM bandwidth) and what it achieved against it."""
+    if flops / (tensor_peak * 1e12) >= nbytes / (hbm_peak * 1e9):
+        ach = flops / (ms / 1e3) / 1e12
+        return dict(bound="tensor", achieved=ach, peak=tensor_peak, unit="TFLOP/s",
+                    frac=ach / tensor_peak, algorithmic_per_launch=flops)
+    ach = nbytes / (ms / 1e3) / 1e9
+    return dict(bound="hbm", achieved=ach, peak=hbm_peak, unit="GB/s", frac=ach / hbm_peak,
+                algorithmic_per_launch=nbytes)
+
+
+def time_calls(call, n, stream, kev=None, local_rank=0):
+    """Time n back-to-back calls on `stream` with CUDA events, sampling the
+    clocks meanwhile; call(i, events) enqueues call i. Returns (ms, clocks)."""
+    import torch
+    clocks = ClockSampler(local_rank)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)
+    t_start.record(stream)
+    for i in range(n):
+        call(i, kev[i].array if kev is not None else None)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    return t_start.elapsed_time(t_end), clk
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -221,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
                                                  forward, _lib, moe_get_device_status,
                                                  quantize_fp8)
     from sparse_mixture_experts_aux_b200.events import KernelEvents
-    from sparse_mixture_experts_aux_b200.inputs import make_inputs, make_x
+    from sparse_mixture_experts_aux_b200.inputs import MIXTRAL_DECODE, make_inputs, make_x
     from oracle import moe_oracle as O  # cpu_baseline leg only
 
     w = workload_by_name(args.workload)
@@ -246,11 +313,12 @@ def run_ours(args, rank, world, local_rank):
         scales = torch.cat(parts)
         torch.cuda.synchronize()
 
-    def call(i, events=None):
-        forward(xs[i % R], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["W_shared"],
-                k=w.k, capacity_factor=w.capacity_factor, router_bias=inp["router_bias"],
-                d_s=w.d_s, workspace=ws, stream=stream, events=events, y=y, aux=aux,
-                counts=counts, weight_scales=scales, act_fp8=act_fp8)
+    def call_on(xlist, yb, i, events=None):
+        forward(xlist[i % len(xlist)], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"],
+                inp["W_shared"], k=w.k, capacity_factor=w.capacity_factor,
+                router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws, stream=stream,
+                events=events, y=yb, aux=aux, counts=counts, weight_scales=scales,
+                act_fp8=act_fp8)
 
     def barrier():
         if world > 1:
@@ -260,26 +328,14 @@ def run_ours(args, rank, world, local_rank):
     kev = [KernelEvents(MOE_NUM_KERNELS) for _ in range(args.steps)]
 
     for i in range(max(3, args.warmup)):
-        call(i)
+        call_on(xs, y, i)
     torch.cuda.synchronize()
     if moe_get_device_status() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
 
-    clocks = ClockSampler(local_rank)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.2)
-    t_start.record(stream)
-    for i in range(args.steps):
-        call(i, kev[i].array)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
+    ms, clk = time_calls(lambda i, ev: call_on(xs, y, i, ev), args.steps, stream, kev, local_rank)
     barrier()
-    ms = t_start.elapsed_time(t_end)
     if moe_get_device_status() != 0:
         raise RuntimeError("device-side wait timed out in the timed region")
     per_kernel = [statistics.mean(kev[i].elapsed_ms(j) for i in range(args.steps))
@@ -288,49 +344,42 @@ def run_ours(args, rank, world, local_rank):
         kv.close()
     ms_max = max_over_ranks(ms, dev)
 
-    # algorithmic work of one step, from this step's own routing counts
-    cnt = counts.cpu().numpy().astype("int64")
-    C = _lib.moe_capacity(w.T, w.E, w.k, w.capacity_factor)
-    C = None if C < 0 else C
-    kept = int(cnt.sum() if C is None else sum(min(int(c), C) for c in cnt))
-    touched = int(sum(1 for c in cnt if (c if C is None else min(int(c), C)) > 0))
-    esz = 2 if w.dtype == "bf16" else 4
-    wsz = 1 if fp8 else esz  # bytes per expert weight (+ 4 per row of scales with FP8)
-    flops_up = 2 * kept * w.d * 2 * w.d_e + (2 * w.T * w.d * 2 * w.d_s if w.d_s else 0)
-    flops_down = 2 * kept * w.d_e * w.d + (2 * w.T * w.d_s * w.d if w.d_s else 0)
-    flops_active = flops_up + flops_down
-    w_bytes = (touched * 3 * w.d * w.d_e * wsz + (touched * 2 * (w.d_e + w.d) * 4 if fp8 else 0)
-               + 3 * w.d * w.d_s * esz + w.E * w.d * 4)
-    act_bytes = 2 * w.T * w.d * esz
+    wk = step_work(w, counts.cpu().numpy().astype("int64"), fp8)
     peaks, peaks_src = load_peaks()
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    if act_fp8:  # E4M3 x E4M3: the bf16 figure times the nominal 4.5 / 2.25 ratio
-        tensor_peak *= 2.0
+    # Headline tensor peak: the burst cuBLAS figure (a kernel timed in a short run at
+    # full clock, as this one is); the sustained, power-capped figure is reported
+    # beside it, labelled. E4M3 x E4M3: the bf16 figures times the nominal 4.5 / 2.25.
+    ratio = 2.0 if act_fp8 else 1.0
+    tensor_peak = peaks["bf16_tflops"] * ratio
+    tensor_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
     hbm_peak = peaks["hbm_gbs"]
 
     ms_step = ms_max / args.steps
     value = job_value(world, w.T, args.steps, ms_max)
-    k_up = per_kernel[4]
-    # the gate/up kernel's own roofline: its FLOPs at tensor peak vs its
-    # algorithmic bytes (touched gate+up weights, permuted rows in, H out) at HBM
-    bytes_up = (touched * 2 * w.d * w.d_e * wsz + (touched * 2 * w.d_e * 4 if fp8 else 0)
-                + (2 * w.d * w.d_s * esz if w.d_s else 0)
-                + (kept + (w.T if w.d_s else 0)) * (w.d + w.d_e) * esz)
-    up_bound = "tensor" if flops_up / (tensor_peak * 1e12) >= bytes_up / (hbm_peak * 1e9) else "hbm"
-    if up_bound == "tensor":
-        achieved, peak, unit, work = flops_up / (k_up / 1e3) / 1e12, tensor_peak, "TFLOP/s", flops_up
-        peak_note = (f"bf16_tflops_sustained x 2 (nominal e4m3/bf16 ratio; of {peaks_src})"
-                     if act_fp8 else f"bf16_tflops_sustained (of {peaks_src})")
-    else:
-        achieved, peak, unit, work = bytes_up / (k_up / 1e3) / 1e9, hbm_peak, "GB/s", bytes_up
-        peak_note = f"hbm_gbs (of {peaks_src})"
+    k_up, k_down = per_kernel[4], per_kernel[5]
+    rl = kernel_roofline(wk["flops_up"], wk["bytes_up"], k_up, tensor_peak, hbm_peak)
+    src = f"bf16_tflops{' x 2 (nominal e4m3/bf16 ratio)' if act_fp8 else ''} (of {peaks_src})"
+    rl["peak_source"] = src if rl["bound"] == "tensor" else f"hbm_gbs (of {peaks_src})"
+    if rl["bound"] == "tensor":
+        rl["frac_of_sustained_peak"] = rl["achieved"] / tensor_sust
+        rl["sustained_peak"] = tensor_sust
+    mhz = (clk or {}).get("sm_mhz")
+    rl["ms_per_launch"] = k_up
+    rl["ms_x_sm_mhz"] = k_up * mhz if mhz else None  # clock-normalised duration
     # DRAM traffic of the dominant kernel: ncu's dram bytes over the algorithmic bytes on a
     # small case of the same kernel and per-expert load, times this launch's algorithmic
-    # bytes (profiles/tc_grouped_gemm_mixtral_shape.md); None where no capture of the
-    # kernel as built stands
+    # bytes; None where no capture of the kernel as built stands
     traffic_ratio = TRAFFIC_RATIO.get((args.workload, args.weights))
-    traffic = traffic_ratio * bytes_up if traffic_ratio is not None else None
-    roofline_ms = max(flops_active / (tensor_peak * 1e12), (w_bytes + act_bytes) / (hbm_peak * 1e9)) * 1e3
+    rl["traffic"] = traffic_ratio * wk["bytes_up"] if traffic_ratio is not None else None
+    rl["traffic_source"] = ("ncu dram bytes / algorithmic bytes = %.3f on the T=1024 E=2 case, "
+                            "times this launch's algorithmic bytes" % traffic_ratio
+                            if traffic_ratio is not None else None)
+    rl = {"kernel": KERNEL_NAMES[4], **rl}
+    rl_down = kernel_roofline(wk["flops_down"], wk["bytes_down"], k_down, tensor_peak, hbm_peak)
+    roof_ms = max(wk["flops"] / (tensor_peak * 1e12),
+                  (wk["w_bytes"] + wk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
+    roof_ms_sust = max(wk["flops"] / (tensor_sust * 1e12),
+                       (wk["w_bytes"] + wk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -338,21 +387,18 @@ def run_ours(args, rank, world, local_rank):
         "dtype": ("e4m3" if act_fp8 else ("bf16" if w.dtype == "bf16" else "f32")),
         "data": "synthetic",
         "config": dict(config_of(w, "inputs larger than L2: %.2f GB of expert weights streamed "
-                                    "per step; x rotates over %d batches" % (w_bytes / 1e9, R)),
+                                    "per step; x rotates over %d batches" % (wk["w_bytes"] / 1e9, R)),
                        weights="e4m3 codes + fp32 row scales" if fp8 else w.dtype,
                        activations="e4m3 rows + fp32 row scales in the experts" if act_fp8
                        else w.dtype),
-        "roofline": {"bound": up_bound, "kernel": KERNEL_NAMES[4], "achieved": achieved,
-                     "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                     "traffic_source": ("ncu dram bytes / algorithmic bytes = %.3f on the "
-                                        "T=1024 E=2 case, times this launch's algorithmic "
-                                        "bytes" % traffic_ratio) if traffic is not None else None,
-                     "algorithmic_per_launch": work, "peak_source": peak_note},
-        "layer": {"active_tflops": flops_active / (ms_step / 1e3) / 1e12,
-                  "active_flops_per_step": flops_active, "touched_weight_bytes": w_bytes,
-                  "roofline_ms": roofline_ms, "frac_of_roofline": roofline_ms / ms_step,
-                  "hbm_gbs_weights": w_bytes / (ms_step / 1e3) / 1e9,
-                  "dropped_fraction": O.dropped_fraction(cnt, C, w.T, w.k),
+        "roofline": rl,
+        "down_roofline": {"kernel": KERNEL_NAMES[5], "ms_per_launch": k_down, **rl_down},
+        "layer": {"active_tflops": wk["flops"] / (ms_step / 1e3) / 1e12,
+                  "active_flops_per_step": wk["flops"], "touched_weight_bytes": wk["w_bytes"],
+                  "roofline_ms": roof_ms, "frac_of_roofline": roof_ms / ms_step,
+                  "frac_of_roofline_sustained_peak": roof_ms_sust / ms_step,
+                  "hbm_gbs_weights": wk["w_bytes"] / (ms_step / 1e3) / 1e9,
+                  "dropped_fraction": O.dropped_fraction(counts.cpu().numpy(), wk["C"], w.T, w.k),
                   "aux": float(aux.cpu()[0])},
         "kernel_ms": {KERNEL_NAMES[j]: per_kernel[j] for j in range(MOE_NUM_KERNELS)},
         # W8A8 adds the x and H quantisers to the 7 kernels of a step
@@ -421,11 +467,64 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        esz = 2 if w.dtype == "bf16" else 4
         line["e2e"] = {"value": job_value(world, w.T, ke, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": w.T * w.d * esz,
                        "d2h_bytes_per_step": w.T * w.d * esz + 4 + 4 * w.E,
                        "steps": ke, "api": "moe_forward_host_io",
                        "streams": NSTR, "host_threads": NSTR}
+        del bufs
+
+    # the weight-streaming decode shape on the same weights: T = 32, one fresh x per call
+    if args.workload == "mixtral" and not args.no_decode and args.decode_calls > 0:
+        wd = MIXTRAL_DECODE.with_(dtype=w.dtype)
+        n = args.decode_calls
+        xd = make_x(wd, str(dev), seed_offset=5000 + 100 * rank, T=wd.T * n).view(n, wd.T, wd.d)
+        yd = torch.empty(wd.T, wd.d, dtype=xd.dtype, device=dev)
+        xl = [xd[i] for i in range(n)]
+        cd = torch.empty(wd.E, dtype=torch.int32, device=dev)
+
+        def dcall(i, events=None):
+            forward(xl[i], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], None, k=wd.k,
+                    workspace=ws, stream=stream, events=events, y=yd, aux=aux, counts=cd,
+                    weight_scales=scales, act_fp8=act_fp8)
+
+        for i in range(max(3, args.warmup)):
+            dcall(i)
+        torch.cuda.synchronize()
+        dkev = [KernelEvents(MOE_NUM_KERNELS) for _ in range(n)]
+        barrier()
+        dms, dclk = time_calls(dcall, n, stream, dkev, local_rank)
+        barrier()
+        if moe_get_device_status() != 0:
+            raise RuntimeError("device-side wait timed out in the decode leg")
+        dk = [statistics.mean(dkev[i].elapsed_ms(j) for i in range(n))
+              for j in range(MOE_NUM_KERNELS)]
+        for kv in dkev:
+            kv.close()
+        dms_max = max_over_ranks(dms, dev)
+        dwk = step_work(wd, cd.cpu().numpy().astype("int64"), fp8)
+        d_ms = dms_max / n
+        d_roof = max(dwk["flops"] / (tensor_peak * 1e12),
+                     (dwk["w_bytes"] + dwk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
+        line["decode"] = {
+            "workload": wd.name, "calls": n, "distinct_x": n, "ms_per_call": d_ms,
+            "tokens_per_s": job_value(world, wd.T, n, dms_max),
+            "touched_weight_bytes": dwk["w_bytes"],
+            "hbm_gbs": (dwk["w_bytes"] + dwk["act_bytes"]) / (d_ms / 1e3) / 1e9,
+            "hbm_peak_gbs": hbm_peak, "roofline_ms": d_roof, "frac_of_roofline": d_roof / d_ms,
+            "gate_up": {"ms_per_launch": dk[4],
+                        **kernel_roofline(dwk["flops_up"], dwk["bytes_up"], dk[4], tensor_peak,
+                                          hbm_peak)},
+            "down": {"ms_per_launch": dk[5],
+                     **kernel_roofline(dwk["flops_down"], dwk["bytes_down"], dk[5], tensor_peak,
+                                       hbm_peak)},
+            "kernel_ms": {KERNEL_NAMES[j]: dk[j] for j in range(MOE_NUM_KERNELS)},
+            "gpu_launches": (MOE_NUM_KERNELS + (2 if act_fp8 else 0)) * n * world,
+            "clocks": dclk,
+            "l2": "weights (%.2f GB) larger than L2; each call reads its own x" % (dwk["w_bytes"] / 1e9),
+        }
+        del xd, xl
 
     # the oracle on the host cores, bounded sample, rank 0 at N=1 only
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -446,8 +545,59 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def main():
-    args = parse_args()
+# --------------------------------------------------------------------------- launch
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_entry(rank, world, port, backend, fn, timeout_s):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    import torch
+    import torch.distributed as dist
+    kw = {}
+    if backend == "nccl":
+        torch.cuda.set_device(rank)
+        kw["device_id"] = torch.device("cuda", rank)
+    dist.init_process_group(backend, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    try:
+        fn(rank, world)
+    finally:
+        dist.destroy_process_group()
+
+
+def launch_local_ranks(n: int, fn, backend: str = "nccl", timeout_s: int = 300) -> list:
+    """Run fn(rank, world) in n spawned processes on this node, one per GPU
+    (LOCAL_RANK = rank), with a process group over `backend` and a rendezvous on
+    127.0.0.1. Returns the processes' exit codes."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_entry, args=(r, n, port, backend, fn, timeout_s))
+             for r in range(n)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout_s + 600)
+        if p.is_alive():
+            p.kill()
+            p.join()
+    return [p.exitcode for p in procs]
+
+
+def run_rank(args, rank, world):
+    """One rank of our arm: run the benchmark, rank 0 prints the line."""
+    line = run_ours(args, rank, world, int(os.environ.get("LOCAL_RANK", rank)))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -456,6 +606,10 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return 0
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        import functools
+        codes = launch_local_ranks(args.gpus, functools.partial(run_rank, args), "nccl")
+        return 0 if all(c == 0 for c in codes) else 1
     import torch
     import torch.distributed as dist
     if world > 1:

@@ -78,6 +78,11 @@ MIXTRAL_PROFILE = Workload("mixtral-shape-profile T=1024 d=4096 E=2 d_e=14336 k=
 # The decode shape with 2 experts (about 0.7 GB of bf16 weights), likewise.
 DECODE_PROFILE = Workload("decode-shape-profile T=32 d=4096 E=2 d_e=14336 k=2",
                           32, 4096, 2, 14336, 2, seed=4)
+# The Mixtral-shaped layer's routing, permute and combine work (T, d, E and k
+# as in the full layer; those kernels do not depend on d_e) with narrow
+# experts, so the whole case holds about 0.2 GB, for hardware-counter captures.
+ROUTING_PROFILE = Workload("routing-kernels-profile T=4096 d=4096 E=8 d_e=256 k=2",
+                           4096, 4096, 8, 256, 2, seed=1)
 
 
 def zipf_router_bias(E: int) -> torch.Tensor:

@@ -1,7 +1,8 @@
 """The multi-rank plumbing of bench.py ("replicas only": no data-path
 collective) on CPU with gloo, world size 2: every rank agrees on the slowest
-rank's time, the job value counts every rank's tokens, and the reference arm
-does its work on rank 0 only."""
+rank's time, the job value counts every rank's tokens, the reference arm
+does its work on rank 0 only, and `--gpus N` without a launcher spawns N
+ranks of its own with a working process group."""
 import datetime
 import os
 import socket
@@ -75,3 +76,25 @@ def test_reference_arm_runs_the_oracle_on_rank0():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _spawned_probe(q, rank, world):
+    import torch
+    import bench
+    ms = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
+    q.put((rank, world, int(os.environ["LOCAL_RANK"]), ms))
+
+
+def test_bench_spawns_its_own_ranks():
+    import functools
+    import multiprocessing
+
+    sys.path.insert(0, ROOT)
+    import bench
+    q = multiprocessing.get_context("spawn").Queue()
+    codes = bench.launch_local_ranks(2, functools.partial(_spawned_probe, q), "gloo",
+                                     timeout_s=60)
+    assert codes == [0, 0]
+    out = sorted(q.get(timeout=30) for _ in range(2))
+    assert [o[:3] for o in out] == [(0, 2, 0), (1, 2, 1)]
+    assert [o[3] for o in out] == [15.0, 15.0]
