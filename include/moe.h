@@ -33,8 +33,13 @@
  *   - Argument errors are detected on the host before anything is enqueued
  *     and return MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE.
  *   - moe_forward is asynchronous on dims->stream; a CUDA launch failure
- *     returns MOE_ERR_CUDA. Bounded device-side waits record a timeout that
- *     moe_get_device_status reports after the caller synchronises.
+ *     returns MOE_ERR_CUDA. Bounded device-side waits record a timeout in two
+ *     places: the call's own status word inside its workspace (see
+ *     moe_workspace_layout_t.status; moe_forward_host_io reports it), and one
+ *     device-wide word that moe_get_device_status reads and clears. The
+ *     device-wide word is shared by every call on the device: with concurrent
+ *     calls (several streams or threads) it cannot tell which call timed out,
+ *     and one caller's read clears it for all. Use the per-call word there.
  *   - Calls on one stream are ordered; two calls that share one workspace
  *     must not overlap on the device.
  */
@@ -61,8 +66,11 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,      /* workspace null, too small or misaligned */
   MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
   MOE_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up (moe_get_device_status) */
-  MOE_ERR_SCRATCH_LIMIT = 6   /* moe_forward_no_alloc: the layer needs more scratch than
+  MOE_ERR_SCRATCH_LIMIT = 6,  /* moe_forward_no_alloc: the layer needs more scratch than
                                  MOE_NO_ALLOC_WORKSPACE_BYTES */
+  MOE_ERR_DEVICE_BOUNDS = 7   /* builds with MOE_DEBUG only: a device-side bounds check on a
+                                 permuted row, a segment start or a TMA row coordinate failed
+                                 (the access was skipped; outputs undefined) */
 } moe_status;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
@@ -206,9 +214,12 @@ MOE_API moe_status moe_forward(const moe_dims* dims,
  * End-to-end variant for callers holding the activations in host memory: the
  * same forward pass, bracketed by the copies. Copies x_host -> x_dev, runs
  * moe_forward, copies y_dev -> y_host, aux_dev -> aux_host and counts_dev ->
- * counts_host, all on dims->stream, then synchronises that stream and returns
- * moe_get_device_status() if the pass itself succeeded. Weights stay device
- * pointers. x_host / y_host should be pinned for full copy bandwidth.
+ * counts_host, all on dims->stream, then synchronises that stream. If the pass
+ * itself was enqueued, it returns MOE_ERR_DEVICE_TIMEOUT when a device-side wait
+ * of this call gave up (read from the call's own status word, so concurrent
+ * calls on other streams do not see each other's timeouts), else MOE_OK.
+ * Weights stay device pointers. x_host / y_host should be pinned for full copy
+ * bandwidth.
  */
 MOE_API moe_status moe_forward_host_io(const moe_dims* dims,
                                const void* x_host, void* x_dev,
@@ -241,14 +252,22 @@ typedef struct {
   size_t xscale;      /* fp32 [rows_max]       scale of each permuted x row */
   size_t hq;          /* uint8 [rows_max, d_e] E4M3 codes of the hidden rows */
   size_t hscale;      /* fp32 [rows_max]       scale of each hidden row */
+  size_t status;      /* int32: this call's status word, 0 when no device-side wait of
+                         this call gave up, nonzero otherwise (valid once the call's
+                         stream has been synchronised; cleared at the start of each call) */
 } moe_workspace_layout_t;
 
 MOE_API moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capacity_factor,
                                 moe_workspace_layout_t* out);
 
-/* Status of the device-side bounded waits since the last call (for the current
- * device); resets it. Call after synchronising the stream(s) used.
- * MOE_OK or MOE_ERR_DEVICE_TIMEOUT (or MOE_ERR_CUDA if it cannot be read). */
+/* Status of the device-side bounded waits (and, in MOE_DEBUG builds, bounds
+ * checks) since the last read, for the current device: reads and clears the
+ * device-wide word in one atomic exchange. Call after synchronising the
+ * stream(s) used. The word is shared by every call on the device; to attribute
+ * a timeout to one of several concurrent calls, read that call's own status
+ * word (moe_workspace_layout_t.status) instead. Returns MOE_OK,
+ * MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, or MOE_ERR_CUDA if it cannot
+ * be read. */
 MOE_API moe_status moe_get_device_status(void);
 
 /* Static, human-readable name of a status code. */
@@ -294,9 +313,13 @@ MOE_API moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales,
  * Instead this call uses one scratch array of MOE_NO_ALLOC_WORKSPACE_BYTES
  * (64 MiB) that lives in the library itself as a statically sized device
  * array: every GPU that loads the library holds it until the process exits.
- * That covers, for example, the Mixtral-shaped layer (d=4096, E=8,
- * d_e=14336, k=2) at T <= 128 tokens per call. The call allocates nothing:
- * no cudaMalloc, no cudaFree, no allocating library routine.
+ * A layer fits when moe_workspace_size() for it is at most
+ * MOE_NO_ALLOC_WORKSPACE_BYTES; that is the test to use. The size grows with
+ * the permuted rows, T*k plus up to 127 padding rows per expert (each
+ * expert's segment is padded to 128 rows), times d and d_e. One example: the
+ * Mixtral-shaped layer (d=4096, E=8, d_e=14336, k=2) fits up to T = 128
+ * tokens per call (about 58 MB). The call allocates nothing: no cudaMalloc,
+ * no cudaFree, no allocating library routine.
  *
  * Arguments and results are exactly those of moe_forward, except that
  * dims->workspace and dims->workspace_bytes are ignored. Inputs and outputs
@@ -308,7 +331,10 @@ MOE_API moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales,
  *
  * Set-up: the first call on each device looks up the device address of the
  * scratch array (cudaGetSymbolAddress) with that device current, and caches
- * it. Make that first call before any stream capture.
+ * it for the life of the process. Make that first call before any stream
+ * capture. Resetting the device (cudaDeviceReset, or tearing down and
+ * re-creating its primary context) after that first call is not supported:
+ * the cached address would be stale.
  *
  * Sharing: every call, on every stream, uses the same scratch array, which
  * keeps the previous call's contents. The pass writes every scratch byte it

@@ -10,6 +10,8 @@ import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# the same library built with MOE_DEBUG (device bounds checks); tests only
+DEBUG_LIB_PATH = os.path.join(_PKG, "libmoe_debug.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -18,6 +20,7 @@ MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_SCRATCH_LIMIT = 6
+MOE_ERR_DEVICE_BOUNDS = 7
 MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
@@ -69,6 +72,7 @@ class moe_workspace_layout_t(ctypes.Structure):
         ("xscale", ctypes.c_size_t),
         ("hq", ctypes.c_size_t),
         ("hscale", ctypes.c_size_t),
+        ("status", ctypes.c_size_t),
     ]
 
 
@@ -79,15 +83,28 @@ class MoeError(RuntimeError):
 
 
 _lib = None
+_debug_lib = None
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     """Load libmoe.so once and declare its signatures. Raises if it is absent."""
     global _lib
-    if _lib is not None:
-        return _lib
+    if _lib is None:
+        _lib = _open(path)
+    return _lib
+
+
+def load_debug() -> ctypes.CDLL:
+    """The MOE_DEBUG build (libmoe_debug.so), loaded once beside the release one."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _open(DEBUG_LIB_PATH)
+    return _debug_lib
+
+
+def _open(path: str) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise RuntimeError(f"libmoe.so not found at {path}; build it with "
+        raise RuntimeError(f"{os.path.basename(path)} not found at {path}; build it with "
                            "`python -m sparse_mixture_experts_aux_b200.build`")
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER
@@ -114,7 +131,6 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_quantize_fp8.restype = i32
     lib.moe_dequantize_fp8.argtypes = [vp, vp, ctypes.c_int64, i32, vp, vp]
     lib.moe_dequantize_fp8.restype = i32
-    _lib = lib
     return lib
 
 

@@ -4,6 +4,9 @@
 
 The library is one translation unit (csrc/moe_api.cu includes the kernel
 headers) linked against the static CUDA runtime; it takes no torch headers.
+--debug builds libmoe_debug.so instead: the same library with MOE_DEBUG, whose
+kernels check permuted rows, segment starts and GEMM tile coordinates against
+their buffers, record a failure in the device error word and skip the access.
 """
 from __future__ import annotations
 
@@ -18,6 +21,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
+DEBUG_LIB = os.path.join(PKG, "libmoe_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -32,20 +36,21 @@ def sources() -> list:
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + [os.path.join(INCLUDE, "moe.h"), os.path.abspath(__file__)]
     return all(os.path.getmtime(s) <= t for s in deps)
 
 
 def build(force: bool = False, debug: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not debug and up_to_date():
-        return LIB
+    out = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(out):
+        return out
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", os.path.join(CSRC, "moe_api.cu")]
+           "-o", out + ".tmp", os.path.join(CSRC, "moe_api.cu")]
     if debug:
         cmd.insert(1, "-DMOE_DEBUG=1")
     if verbose_ptxas:
@@ -55,8 +60,8 @@ def build(force: bool = False, debug: bool = False, verbose_ptxas: bool = False)
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose_ptxas:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

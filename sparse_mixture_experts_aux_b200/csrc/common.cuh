@@ -6,10 +6,24 @@
 
 namespace moe {
 
-// Device-side error word, read and cleared by moe_get_device_status().
+// Device-side error word of this device, shared by every call on it; read and
+// cleared in one atomic exchange by moe_get_device_status(). Each call also has
+// a status word of its own in its workspace (cleared by the scan kernel, set by
+// a GEMM CTA that gave up), which attributes a timeout to the call that hit it.
 // Bit 0: an mbarrier wait in a GEMM kernel gave up after its time limit.
+// Bit 1 (builds with MOE_DEBUG only): a device-side bounds check failed and
+// the access was skipped.
 __device__ int g_dev_error;
+__device__ int g_dev_error_taken;  // the value the last exchange took out
 constexpr int DEVERR_TIMEOUT = 1;
+constexpr int DEVERR_BOUNDS = 2;
+
+// Read and clear the device error word in one step, so that a bit set by a
+// kernel between a separate read and clear cannot be lost.
+__global__ void take_device_error_kernel() { g_dev_error_taken = atomicExch(&g_dev_error, 0); }
+
+// Record a failed bounds check (MOE_DEBUG builds).
+__device__ __forceinline__ void flag_bounds() { atomicOr(&g_dev_error, DEVERR_BOUNDS); }
 
 // Rows of the permuted buffers are grouped per expert in segments padded to
 // this many rows, so that no GEMM M-tile straddles two experts.

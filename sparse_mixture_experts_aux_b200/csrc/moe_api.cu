@@ -37,7 +37,7 @@ struct Plan {
   bool router_narrow;  // few experts, many tokens: warp-per-token-group router kernel
   int64_t rows_max;
   size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
-      o_tile_start, o_pair_start, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys,
+      o_tile_start, o_pair_start, o_status, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys,
       // E4M3 activations (MOE_WEIGHTS_FP8_W8A8): x codes and scales per token,
       // scales of the permuted x rows, H codes and scales per permuted row
       o_xq, o_sx, o_xsc, o_hq, o_hsc, total;
@@ -116,6 +116,7 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   p.o_probsum = take(static_cast<size_t>(E) * 8);
   p.o_tile_start = take(static_cast<size_t>(E + 1) * 4);
   p.o_pair_start = take(static_cast<size_t>(E + 1) * 4);
+  p.o_status = take(4);  // the call's own device status word
   p.o_rowgate = take(R * 4);
   p.o_xp = take(R * p.d * p.esz);
   p.o_h = take(R * p.de * p.esz);
@@ -404,7 +405,8 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   tm.at(4);
   moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk, P.E,
                                        P.T, P.k, P.C, counts, base, tile_start, pair_start,
-                                       probsum, aux);
+                                       probsum, aux, reinterpret_cast<int*>(ws + P.o_status),
+                                       P.rows_max);
   tm.at(5);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
 
@@ -424,14 +426,15 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
       dim3 qgrid((T + 7) / 8, (qvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
       moe::scatter_kernel<uint8_t><<<qgrid, 256, 0, st>>>(
           xq, P.d, T, P.k, P.E, P.C, idx, gate, lrank, base, tile_start, slot, rowgate,
-          reinterpret_cast<uint8_t*>(xp), sx, reinterpret_cast<float*>(ws + P.o_xsc));
+          reinterpret_cast<uint8_t*>(xp), P.rows_max, sx, reinterpret_cast<float*>(ws + P.o_xsc));
     } else if (dims->weight_format == MOE_WEIGHTS_FP8) {  // the FP8-weight GEMMs read fp16 rows
       moe::scatter_kernel<TX, true><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate,
                                                           lrank, base, tile_start, slot, rowgate,
-                                                          xp);
+                                                          xp, P.rows_max);
     } else
       moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
-                                                    base, tile_start, slot, rowgate, xp);
+                                                    base, tile_start, slot, rowgate, xp,
+                                                    P.rows_max);
   }
   tm.at(7);
   return launched();
@@ -482,6 +485,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   int32_t* slot = reinterpret_cast<int32_t*>(ws + P.o_slot);
   int32_t* tile_start = reinterpret_cast<int32_t*>(ws + P.o_tile_start);
   float* rowgate = reinterpret_cast<float*>(ws + P.o_rowgate);
+  int* call_err = reinterpret_cast<int*>(ws + P.o_status);
+  const int rows_cap = static_cast<int>(P.rows_max);  // permuted rows (debug bounds checks)
 
   if (P.bf16) {
     using bf16 = __nv_bfloat16;
@@ -523,13 +528,15 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tu.num_groups = 1;
       tu.timeout_ns = wait_tmo;
       tu.drain_timeout_ns = kDrainTimeoutNs;
-      tu.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+      tu.call_err = call_err;
+      tu.g[0] = {tile_start, E, rows_cap, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
                  (P.d + K8 - 1) / K8, P.de, h, nullptr, xsc, sc, sc + gsz, P.de};
       moe::tc::TcParams td{};
       td.num_groups = 1;
       td.timeout_ns = wait_tmo;
       td.drain_timeout_ns = kDrainTimeoutNs;
-      td.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, (P.de + K8 - 1) / K8,
+      td.call_err = call_err;
+      td.g[0] = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN, (P.de + K8 - 1) / K8,
                  P.d, yrows, rowgate, hsc, sc + 2 * gsz, sc + 2 * gsz, P.d};
       tm.at(8);
       launch_tc<moe::tc::EPI_SWIGLU_TC, true>(arows, num_sms, st, up, tu);
@@ -560,7 +567,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       moe::tcf8::F8Params fu{};
       fu.timeout_ns = wait_tmo;
       fu.drain_timeout_ns = kDrainTimeoutNs;
-      fu.grp.g = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+      fu.call_err = call_err;
+      fu.grp.g = {tile_start, E, rows_cap, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
                   P.d / moe::tc::BK, P.de, h, nullptr};
       fu.grp.scale0 = sc;
       fu.grp.scale1 = sc + gsz;
@@ -568,7 +576,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       moe::tcf8::F8Params fd{};
       fd.timeout_ns = wait_tmo;
       fd.drain_timeout_ns = kDrainTimeoutNs;
-      fd.grp.g = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
+      fd.call_err = call_err;
+      fd.grp.g = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
                   P.d, yrows, rowgate};
       fd.grp.scale0 = sc + 2 * gsz;
       fd.grp.scale1 = sc + 2 * gsz;
@@ -622,7 +631,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         tu.num_groups = ng;
         tu.timeout_ns = wait_tmo;
         tu.drain_timeout_ns = kDrainTimeoutNs;
-        tu.g[0] = {tile_start, pair_start, E, 0, (P.de + BNp / 2 - 1) / (BNp / 2),
+        tu.call_err = call_err;
+        tu.g[0] = {tile_start, pair_start, E, rows_cap, (P.de + BNp / 2 - 1) / (BNp / 2),
                    P.d / moe::tc::BK, P.de, h, nullptr};
         if (P.ds)
           tu.g[1] = {nullptr, nullptr, 1, T, (P.ds + BNp / 2 - 1) / (BNp / 2), P.d / moe::tc::BK,
@@ -636,7 +646,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         tp.num_groups = ng;
         tp.timeout_ns = wait_tmo;
         tp.drain_timeout_ns = kDrainTimeoutNs;
-        tp.g[0] = {tile_start, E, 0, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
+        tp.call_err = call_err;
+        tp.g[0] = {tile_start, E, rows_cap, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
                    P.d / moe::tc::BK, P.de, h, nullptr};
         if (P.ds)
           tp.g[1] = {nullptr, 1, T, (P.ds + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
@@ -665,7 +676,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         td.num_groups = ng;
         td.timeout_ns = wait_tmo;
         td.drain_timeout_ns = kDrainTimeoutNs;
-        td.g[0] = {tile_start, pair_start, E, 0, (P.d + BNp - 1) / BNp, P.de / moe::tc::BK, P.d,
+        td.call_err = call_err;
+        td.g[0] = {tile_start, pair_start, E, rows_cap, (P.d + BNp - 1) / BNp, P.de / moe::tc::BK, P.d,
                    yrows, rowgate};
         if (P.ds)
           td.g[1] = {nullptr, nullptr, 1, T, (P.d + BNp - 1) / BNp, P.ds / moe::tc::BK, P.d, ys,
@@ -679,7 +691,8 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         tp.num_groups = ng;
         tp.timeout_ns = wait_tmo;
         tp.drain_timeout_ns = kDrainTimeoutNs;
-        tp.g[0] = {tile_start, E, 0, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
+        tp.call_err = call_err;
+        tp.g[0] = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
                    P.d, yrows, rowgate};
         if (P.ds)
           tp.g[1] = {nullptr, 1, T, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.ds / moe::tc::BK,
@@ -696,7 +709,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       const int nvec = P.d * 2 / 16;
       dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
       moe::combine_kernel<bf16><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
-                                                      static_cast<bf16*>(y));
+                                                      static_cast<bf16*>(y), P.rows_max);
     }
     tm.at(13);
     return launched();
@@ -744,7 +757,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     const int nvec = P.d * 4 / 16;
     dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
     moe::combine_kernel<float><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
-                                                     static_cast<float*>(y));
+                                                     static_cast<float*>(y), P.rows_max);
   }
   tm.at(13);
   return launched();
@@ -784,6 +797,7 @@ moe_status moe_workspace_layout(const moe_dims* dims, int E, int k, float capaci
   out->xscale = P.o_xsc;
   out->hq = P.o_hq;
   out->hscale = P.o_hsc;
+  out->status = P.o_status;
   return MOE_OK;
 }
 
@@ -795,14 +809,15 @@ moe_status moe_forward(const moe_dims* dims, const void* x, const float* W_r, co
 }
 
 moe_status moe_get_device_status(void) {
+  // one atomic exchange on the device takes the word out and clears it; the
+  // synchronous copy on the legacy default stream then reads what it took
+  moe::take_device_error_kernel<<<1, 1>>>();
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, moe::g_dev_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(moe::g_dev_error, &zero, sizeof(int)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    return MOE_ERR_DEVICE_TIMEOUT;
-  }
+  if (cudaMemcpyFromSymbol(&v, moe::g_dev_error_taken, sizeof(int)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (v & moe::DEVERR_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
+  if (v & moe::DEVERR_BOUNDS) return MOE_ERR_DEVICE_BOUNDS;
   return MOE_OK;
 }
 
@@ -829,22 +844,18 @@ moe_status moe_forward_host_io(const moe_dims* dims, const void* x_host, void* x
       cudaMemcpyAsync(counts_host, counts_dev, sizeof(int32_t) * E, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  // the status word is read in order on this stream (a synchronous symbol copy
-  // would wait on the legacy default stream and so on other callers' work)
+  // this call's own status word (in its workspace), read in order on its stream:
+  // concurrent callers on other streams neither wait on it nor see its timeouts
   int v = 0;
-  if (cudaMemcpyFromSymbolAsync(&v, moe::g_dev_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
-                                st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbolAsync(moe::g_dev_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
-                                st) != cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
+  if (dims->T > 0) {
+    const Plan P = make_plan(dims, E, k, capacity_factor);
+    const uint8_t* ws = static_cast<const uint8_t*>(dims->workspace);
+    if (cudaMemcpyAsync(&v, ws + P.o_status, sizeof(int), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
       return MOE_ERR_CUDA;
-    return MOE_ERR_DEVICE_TIMEOUT;
   }
-  return MOE_OK;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  return v != 0 ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
 }
 
 const char* moe_status_string(moe_status s) {
@@ -856,6 +867,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
     case MOE_ERR_SCRATCH_LIMIT: return "MOE_ERR_SCRATCH_LIMIT";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS";
   }
   return "MOE_STATUS_UNKNOWN";
 }

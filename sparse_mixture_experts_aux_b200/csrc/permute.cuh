@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ gate,
     const int32_t* __restrict__ lrank, const int32_t* __restrict__ base,
     const int32_t* __restrict__ tile_start, int32_t* __restrict__ slot_pos,
-    float* __restrict__ row_gate, TX* __restrict__ xp,
+    float* __restrict__ row_gate, TX* __restrict__ xp, int64_t rows_max,
     const float* __restrict__ scale_in = nullptr, float* __restrict__ scale_out = nullptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -61,6 +61,14 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int e = idx[a];
     const int rank = base[(size_t)(t / ROUTE_CHUNK) * E + e] + lrank[a];
     if (C < 0 || (int64_t)rank < C) mypos = tile_start[e] * ROW_TILE + rank;
+#if defined(MOE_DEBUG)
+    // the row must lie inside its expert's segment and the permuted buffers
+    if (mypos >= 0 && ((int64_t)mypos >= rows_max || mypos >= tile_start[e + 1] * ROW_TILE ||
+                       e < 0 || e >= E)) {
+      flag_bounds();
+      mypos = -1;
+    }
+#endif
     if (blockIdx.y == 0) {
       if (mypos >= 0) {
         row_gate[mypos] = gate[a];
@@ -91,12 +99,20 @@ __global__ void __launch_bounds__(256) scatter_kernel(
 template <typename TY>
 __global__ void __launch_bounds__(256) combine_kernel(
     const TY* __restrict__ yrows, const TY* __restrict__ ys, const int32_t* __restrict__ slot_pos,
-    int T, int k, int d, TY* __restrict__ y) {
+    int T, int k, int d, TY* __restrict__ y, int64_t rows_max) {
   constexpr int VN = Vec16<TY>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;  // warp-uniform
-  const int mypos = (lane < k) ? slot_pos[(size_t)t * k + lane] : -1;
+  int mypos = (lane < k) ? slot_pos[(size_t)t * k + lane] : -1;
+#if defined(MOE_DEBUG)
+  if ((int64_t)mypos >= rows_max) {  // a permuted row outside the buffers
+    flag_bounds();
+    mypos = -1;
+  }
+#else
+  (void)rows_max;
+#endif
   const int nvec = (int)((size_t)d * sizeof(TY) / 16);
   const int c_begin = blockIdx.y * PERMUTE_CHUNK_VECS;
   const int c_end = c_begin + PERMUTE_CHUNK_VECS < nvec ? c_begin + PERMUTE_CHUNK_VECS : nvec;

@@ -659,15 +659,18 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
 //   pair_start   = exclusive scan of ceil(segment tiles / 2) (CTA-pair tiles)
 //   probsum[e]   = sum of the probability partials, fp64, fixed order
 //   aux          = E * sum_e (counts_e / (T k)) (probsum_e / T), fp64, fixed tree
+// and clears the call's status word.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) scan_kernel(
     const int32_t* __restrict__ hist, int nblk, const double* __restrict__ psum_part, int nparts,
     int E, int64_t T, int k, int64_t C, int32_t* __restrict__ counts, int32_t* __restrict__ base,
     int32_t* __restrict__ tile_start, int32_t* __restrict__ pair_start,
-    double* __restrict__ probsum, float* __restrict__ aux) {
+    double* __restrict__ probsum, float* __restrict__ aux, int* __restrict__ call_err,
+    int64_t rows_max) {
   __shared__ int s_scan[2][1024];
   __shared__ double s_sum[1024];
   const int e = threadIdx.x;
+  if (e == 0 && call_err != nullptr) *call_err = 0;  // the GEMMs of this call run after this
   int tiles = 0;
   double term = 0.0;
   if (e < E) {
@@ -697,7 +700,12 @@ __global__ void __launch_bounds__(1024) scan_kernel(
     __syncthreads();
   }
   if (e < E) tile_start[e] = s_scan[cur][e] - tiles;
-  if (e == E - 1) tile_start[E] = s_scan[cur][e];
+  if (e == E - 1) {
+    tile_start[E] = s_scan[cur][e];
+#if defined(MOE_DEBUG)
+    if ((int64_t)s_scan[cur][e] * ROW_TILE > rows_max) flag_bounds();  // segments overflow
+#endif
+  }
   // the same scan over pairs of tiles (a CTA pair computes two tiles of one expert)
   const int pairs = (tiles + 1) / 2;
   __syncthreads();

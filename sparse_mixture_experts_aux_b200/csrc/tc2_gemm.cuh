@@ -53,7 +53,8 @@ struct Tc2Group {
   const int32_t* tile_start;  // routed: [E+1] segment starts in 128-row tiles; NULL = dense
   const int32_t* pair_start;  // routed: [E+1] exclusive scan of ceil(tiles_e / 2)
   int E;
-  int rows;                   // dense groups: valid rows
+  int rows;                   // dense groups: valid rows; routed groups: rows of the permuted
+                              // buffers (the bounds checks of MOE_DEBUG builds)
   int n_tiles;                // output tiles per expert along N
   int k_blocks;               // K / BK
   int N;                      // output columns
@@ -66,6 +67,7 @@ struct Tc2Params {
   int num_groups;
   unsigned long long timeout_ns;
   unsigned long long drain_timeout_ns;
+  int* call_err;  // the call's own status word (NULL: none)
 };
 
 // ----------------------------------------------------------------------------
@@ -218,6 +220,21 @@ __device__ __forceinline__ PairTile decode_pair(long long tile, long long tiles0
   return t;
 }
 
+// Builds with MOE_DEBUG: a pair tile whose expert, N block or rows fall outside
+// the buffers (routed: both CTAs' rows when the second half is valid, else the
+// first CTA's; dense: the first row). Release builds: false.
+__device__ __forceinline__ bool pair_out_of_bounds(const PairTile& t, const Tc2Group& g) {
+#if defined(MOE_DEBUG)
+  if (t.nb < 0 || t.nb >= g.n_tiles || t.row0 < 0) return true;
+  if (g.tile_start != nullptr)
+    return t.e < 0 || t.e >= g.E || t.row0 + HALF_M * (t.half_valid[1] ? 2 : 1) > g.rows;
+  return t.row0 >= g.rows;
+#else
+  (void)t; (void)g;
+  return false;
+#endif
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const Tc2Params p) {
@@ -300,6 +317,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = cluster_id; ok && tile < total; tile += num_clusters) {
         const PairTile ti = decode_pair(tile, tiles0, p, s_ts, s_ps);
+        if (pair_out_of_bounds(ti, p.g[ti.g])) {
+          flag_bounds();
+          continue;
+        }
         const int kbs = p.g[ti.g].k_blocks;
         const int arow = ti.row0 + HALF_M * (int)rank;
         for (int kb = 0; kb < kbs; ++kb) {
@@ -328,7 +349,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         aborted = true;
         if (leader)  // phases the leader armed complete once both CTAs' bytes land
           for (int s = 0; s < STAGES; ++s)
-            if ((issued >> s) & 1u) tc::wait_drain(full_bar(s), (last_par >> s) & 1u, drain_tmo);
+            if ((issued >> s) & 1u)
+              tc::wait_drain(full_bar(s), (last_par >> s) & 1u, abort_flag, drain_tmo);
       }
     }
   } else if (warp == 1) {
@@ -340,6 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = cluster_id; ok && tile < total; tile += num_clusters) {
         const PairTile ti = decode_pair(tile, tiles0, p, s_ts, s_ps);
+        if (pair_out_of_bounds(ti, p.g[ti.g])) continue;
         const int kbs = p.g[ti.g].k_blocks;
         if (!wait_pair(tempty_bar(acc), acc_phase ^ 1u, abort_flag, peer_abort, tmo)) {
           ok = false;
@@ -369,7 +392,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) aborted = true;
       tc_commit_pair(done_bar);
-      tc::wait_drain(done_bar, 0u, drain_tmo);
+      tc::wait_drain(done_bar, 0u, abort_flag, drain_tmo);
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
@@ -380,6 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (long long tile = cluster_id; tile < total; tile += num_clusters) {
       const PairTile ti = decode_pair(tile, tiles0, p, s_ts, s_ps);
       const Tc2Group& g = p.g[ti.g];
+      if (pair_out_of_bounds(ti, g)) continue;
       int ok = 1;
       if (lane == 0)
         ok = wait_pair(tfull_bar(acc), acc_phase, abort_flag, peer_abort, tmo) ? 1 : 0;
@@ -451,6 +475,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   cluster_sync();  // the leader's MMAs into this CTA's TMEM have completed
   tc::tc_fence_after();
+  tc::record_call_status(abort_flag, p.call_err);
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);

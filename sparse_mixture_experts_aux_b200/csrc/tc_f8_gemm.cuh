@@ -1,14 +1,22 @@
-// Grouped expert GEMMs with FP8 (E4M3) expert weights, dequantised on chip.
+// Grouped expert GEMMs with quantised expert weights, dequantised on chip:
+// FP8 (E4M3 codes, one fp32 scale per output row) or MXFP4 (E2M1 codes packed
+// two per byte, one power-of-two E8M0 scale per 32 weights along K, and a
+// per-row fp32 factor 2^(the row's largest block exponent)).
 //
-// The weights stay in HBM as E4M3 codes with one fp32 scale per output row,
-// so a weight-streaming (decode) pass reads half the bytes of bf16 weights.
+// The weights stay in HBM as codes, so a weight-streaming (decode) pass reads
+// half (FP8) or about a quarter (MXFP4: 4.25 bits per weight) of the bytes of
+// bf16 weights. MXFP4 codes decode to fp16 exactly with one instruction per
+// pair; each is then multiplied in fp16 by 2^(X_block - X_row), a power of two,
+// which is exact while X_block >= X_row - 23, and the row factor 2^X_row
+// multiplies the fp32 accumulator in the epilogue like the FP8 row scale.
 // The MMAs run kind::f16 with fp16 operands: E4M3 codes convert to fp16 exactly
 // with one instruction per pair, the permuted activations arrive as fp16 (the
 // scatter kernel converts them; exact for 2^-14 <= |x| <= 65504, saturating
 // above), and this kernel stores H as fp16. Three shared-memory rings:
-//   Q  FP8 weight tiles, 256 rows x 128 codes (two 64-deep K chunks, full
-//      128-byte lines, 128-byte swizzle); TMA in, released by the converter
-//      warps once decoded, so the weight stream never waits for the MMAs
+//   Q  weight code tiles, 256 rows x 128 bytes (FP8: 128 codes, two 64-deep K
+//      chunks; MXFP4: 256 codes, four chunks), full 128-byte lines, 128-byte
+//      swizzle; TMA in, released by the converter warps once decoded, so the
+//      weight stream never waits for the MMAs
 //   A  stages of CH fp16 activation boxes (TMA), released by the MMA commit;
 //      deeper than S, so the boxes (L2 hits) are fetched well ahead
 //   S  stages of CH decoded fp16 weight tiles (256 x 64 each, the
@@ -34,7 +42,9 @@
 //   tfull/tempty/done as in the bf16 kernel.
 #pragma once
 #include "tc_gemm.cuh"
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
+#include <limits.h>
 
 namespace moe {
 namespace tcf8 {
@@ -53,19 +63,27 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int BAR_BYTES = 256;
 constexpr int CONV_WARP0 = 6;
 
-template <int AR>
+enum { WQ_FP8 = 0, WQ_MXFP4 = 1 };
+
+// Ring shape for an activation box of AR rows and weight format WQ. For small
+// boxes (weight-streaming shapes) a stage is one 64-deep chunk and the code
+// ring is four deep, so up to 128 KB of codes per SM are in flight while the
+// decoded tiles turn over; for 128-row boxes the decoded ring is deeper.
+template <int AR, int WQ = WQ_FP8>
 struct F8Shape {
   static_assert(AR == 128 || AR == 64 || AR == 32, "activation box rows");
-  static constexpr int CH = AR == 128 ? 1 : 2;       // 64-deep K chunks per stage
+  static constexpr int CH = 1;                       // 64-deep K chunks per stage
   static constexpr int A_SUB = AR * BK * 2;          // fp16 activation box of one chunk
   static constexpr int B_SUB = BN * BK * 2;          // decoded fp16 weights of one chunk
   static constexpr int A_BYTES = CH * A_SUB;         // a stage of ring A
   static constexpr int S_BYTES = CH * B_SUB;         // a stage of ring S (weights)
-  static constexpr int QK = 2 * BK;                  // codes per weight row in a Q stage
-  static constexpr int Q_BYTES = BN * QK;            // 256 rows x 128 B
+  static constexpr int Q_ROW = 128;                  // bytes per weight row in a Q stage
+  static constexpr int QK = WQ == WQ_MXFP4 ? 256 : 128;  // codes per weight row in a Q stage
+  static constexpr int QCH = QK / BK;                // 64-deep chunks per Q stage
+  static constexpr int Q_BYTES = BN * Q_ROW;         // 256 rows x 128 B
   static constexpr int NS = AR == 128 ? 3 : 2;
-  static constexpr int NA = AR == 64 ? 2 : 4;        // activations run ahead of the weights
-  static constexpr int NQ = 2;
+  static constexpr int NA = 4;                       // activations run ahead of the weights
+  static constexpr int NQ = AR == 128 ? 2 : 4;
   static constexpr int RING_BYTES = NS * S_BYTES + NA * A_BYTES + NQ * Q_BYTES;
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
@@ -81,12 +99,18 @@ struct F8Group {
   const float* scale0;     // per output row of the weight: gate (SwiGLU) or down scales
   const float* scale1;     // up scales (SwiGLU)
   int64_t scale_stride;    // floats between experts
+  // MXFP4 only: E8M0 block exponents (biased by 127), [rows][K / 32] per expert
+  const uint8_t* bscale0;  // gate (SwiGLU) or down
+  const uint8_t* bscale1;  // up (SwiGLU)
+  int64_t bscale_stride;   // bytes between experts
+  int kblk;                // bytes per weight row (K / 32)
 };
 
 struct F8Params {
   F8Group grp;
   unsigned long long timeout_ns;
   unsigned long long drain_timeout_ns;
+  int* call_err;  // the call's own status word (NULL: none)
 };
 
 // Four E4M3 codes (code i in byte i of `w`) -> four fp16 values, as two f16x2
@@ -101,6 +125,39 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32
       "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(w));
+}
+
+// Eight E2M1 codes (two per byte, the even element in the low nibble) -> eight
+// fp16 values as four f16x2 words, with the hardware conversion: one
+// instruction per pair, exact (every E2M1 value is an fp16 value).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t* o) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// The fp16 multiplier 2^(X - 127) / row_factor of one MXFP4 block: a power of
+// two when the row factor is one (2^X_row), exact in fp16 down to 2^-24.
+__device__ __forceinline__ uint32_t mx_block_multiplier(uint32_t e8m0, float inv_row_factor) {
+  const float m = ldexpf(inv_row_factor, (int)e8m0 - 127);
+  const __half2 h = __float2half2_rn(m);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Sixteen MXFP4 codes (8 bytes) of one block -> sixteen fp16 values
+// code * multiplier, as eight f16x2 words.
+__device__ __forceinline__ void mxfp4x16_to_f16x16(uint2 c, uint32_t mult, uint32_t* o) {
+  e2m1x8_to_f16x8(c.x, o);
+  e2m1x8_to_f16x8(c.y, o + 4);
+  const __half2 m = *reinterpret_cast<const __half2*>(&mult);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __half2 v = *reinterpret_cast<const __half2*>(&o[i]);
+    v = __hmul2(v, m);
+    o[i] = *reinterpret_cast<const uint32_t*>(&v);
+  }
 }
 
 // fp32 pair -> f16x2, saturating at +-65504 (H of the FP8-weight path).
@@ -139,10 +196,10 @@ __device__ __forceinline__ tc::TileInfo decode_tile_f8(long long tile, const tc:
 }
 
 
-template <int EPI, int AR>
+template <int EPI, int AR, int WQ = WQ_FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_f8_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const F8Params p) {
-  using Sh = F8Shape<AR>;
+  using Sh = F8Shape<AR, WQ>;
   constexpr int NS = Sh::NS, NA = Sh::NA, NQ = Sh::NQ, CH = Sh::CH;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = tc::smem_addr(smem_raw);
@@ -207,7 +264,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const long long total = (long long)G.n_tiles * s_ts[G.E];
   const int nck = G.k_blocks;                 // 64-deep K chunks per tile
   const int nst = (nck + CH - 1) / CH;        // S stages per tile
-  const int nqs = (nck + 1) / 2;              // Q stages per tile
+  const int nqs = (nck + Sh::QCH - 1) / Sh::QCH;  // Q stages per tile
   const unsigned long long tmo = p.timeout_ns, drain_tmo = p.drain_timeout_ns;
 
   if (warp == 0) {
@@ -219,6 +276,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+        if (tc::tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, G)) {
+          flag_bounds();
+          continue;
+        }
         for (int st = 0; st < nst; ++st) {
           if (!tc::wait_bounded(aempty(as), aph ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const int nv = min(CH, nck - st * CH);
@@ -233,7 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok)  // let every copy already issued land before the CTA exits
         for (int i = 0; i < NA; ++i)
-          if ((issued >> i) & 1u) tc::wait_drain(afull(i), (par >> i) & 1u, drain_tmo);
+          if ((issued >> i) & 1u) tc::wait_drain(afull(i), (par >> i) & 1u, abort_flag, drain_tmo);
     }
   } else if (warp == QPROD_WARP) {
     // ---------------------------------------------------------- weight producer
@@ -245,10 +306,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+        if (tc::tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, G)) continue;
         for (int qi = 0; qi < nqs; ++qi) {
           if (!tc::wait_bounded(qempty(qs), qph ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const uint32_t dq = q_0 + qs * Sh::Q_BYTES;
-          const int x = qi * (Sh::QK / 4);  // the codes are described as 32-bit words
+          const int x = qi * (Sh::Q_ROW / 4);  // the codes are described as 32-bit words
           tc::mbar_expect_tx(qfull(qs), Sh::Q_BYTES);
           if (EPI == tc::EPI_SWIGLU_TC) {
             tc::tma_load_3d(dq, &maps.b0[0], qfull(qs), x, ti.nb * (BN / 2), ti.e);
@@ -264,7 +326,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok)
         for (int i = 0; i < NQ; ++i)
-          if ((issued >> i) & 1u) tc::wait_drain(qfull(i), (par >> i) & 1u, drain_tmo);
+          if ((issued >> i) & 1u) tc::wait_drain(qfull(i), (par >> i) & 1u, abort_flag, drain_tmo);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -274,6 +336,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t sph = 0, aph = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+#if defined(MOE_DEBUG)
+        const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+        if (tc::tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, G)) continue;
+#endif
         if (!tc::wait_bounded(tempty(acc), acc_phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -300,27 +366,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (acc == 0u) acc_phase ^= 1u;
       }
       tc::tc_commit(done_bar);
-      tc::wait_drain(done_bar, 0u, drain_tmo);
+      tc::wait_drain(done_bar, 0u, abort_flag, drain_tmo);
     }
   } else if (warp >= CONV_WARP0 && warp < CONV_WARP0 + CONV_WARPS) {
     // ---------------------------------------------------------------- converters
-    // For chunk g, 256 threads turn half (g & 1) of the Q tile (chunks 4h..4h+3
-    // of each 128-byte row, stored at chunk ^ (row & 7)) into the fp16 tile: 16
-    // codes -> two 16-byte chunks at (2c, 2c+1) ^ (row & 7). A thread owns rows
-    // r, r+64, r+128, r+192 with r & 7 = its lane & 7, so the 8 lanes of every
-    // shared-memory phase hit 8 different 16-byte bank groups, both when reading
-    // and when writing.
+    // For chunk g, 256 threads turn part h = g % QCH of the Q tile into the
+    // fp16 tile (the 128-byte rows are stored with 16-byte chunk j at
+    // j ^ (row & 7)). FP8: 16 codes (16-byte chunk 4h + c4) -> two 16-byte
+    // chunks at (2c, 2c+1) ^ (row & 7). MXFP4: 16 codes (the 8-byte half
+    // c4 & 1 of 16-byte chunk 2h + c4/2, one 32-weight block shared by two
+    // threads) -> the same two chunks. A thread owns rows r, r+64, r+128, r+192
+    // with r & 7 = its lane & 7, so the 8 lanes of every shared-memory phase
+    // hit 8 different 16-byte bank groups, both when reading and when writing.
     const int ct = threadIdx.x - CONV_WARP0 * 32;
     const int r_lo = ct & 7, c4 = (ct >> 3) & 3, r_hi = ct >> 5;
     const int row0 = r_hi * 8 + r_lo;  // 0..63
     const int pos0 = ((2 * c4) ^ r_lo) << 4, pos1 = ((2 * c4 + 1) ^ r_lo) << 4;
-    const uint32_t q_row = row0 * Sh::QK;
+    const uint32_t q_row = row0 * Sh::Q_ROW;
     const uint32_t b_row = r_hi * 1024 + r_lo * 128;
     const bool first = warp == CONV_WARP0;
     int ss = 0, qs = 0, as = 0;
     uint32_t sph = 0, qph = 0, aph = 0;
     bool ok = true;
+    // MXFP4: per owned row, its block exponents (this Q stage's eight, and the
+    // next stage's, loaded one stage ahead) and 1 / its row factor
+    const uint8_t* bsrow[4] = {nullptr, nullptr, nullptr, nullptr};
+    float inv_rf[4] = {0.f, 0.f, 0.f, 0.f};
+    uint2 bs_cur[4], bs_nxt[4];
+    auto load_bs = [&](int qi) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        bs_nxt[i] = bsrow[i] != nullptr
+                        ? __ldg(reinterpret_cast<const uint2*>(bsrow[i] + (size_t)qi * 8))
+                        : make_uint2(0u, 0u);
+    };
     for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+#if defined(MOE_DEBUG)
+      {
+        const tc::TileInfo td = decode_tile_f8(tile, G, s_ts);
+        if (tc::tile_out_of_bounds(td.e, td.nb, td.row0, BM, G)) continue;
+      }
+#endif
+      if constexpr (WQ == WQ_MXFP4) {
+        const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = row0 + 64 * i;  // row of the 256-row weight tile
+          const bool up = EPI == tc::EPI_SWIGLU_TC && rr >= BN / 2;
+          const int grow = EPI == tc::EPI_SWIGLU_TC ? ti.nb * (BN / 2) + (rr & (BN / 2 - 1))
+                                                    : ti.nb * BN + rr;
+          const bool valid = grow < G.N;  // rows past N are zero-filled by TMA
+          const uint8_t* bs = up ? p.grp.bscale1 : p.grp.bscale0;
+          const float* rf = up ? p.grp.scale1 : p.grp.scale0;
+          bsrow[i] = valid ? bs + (int64_t)ti.e * p.grp.bscale_stride + (int64_t)grow * p.grp.kblk
+                           : nullptr;
+          inv_rf[i] = valid ? 1.0f / __ldg(rf + (int64_t)ti.e * p.grp.scale_stride + grow) : 0.f;
+        }
+        load_bs(0);
+      }
       for (int st = 0; st < nst; ++st) {
         // lane 0 waits (bounded) for the stage's slot to be free; __syncwarp
         // then orders the other lanes' writes after it
@@ -329,11 +432,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
         const int nv = min(CH, nck - st * CH);
         uint8_t* const bst = s_base + ss * Sh::S_BYTES + b_row;
-        // all of this stage's codes are loaded before any is decoded (two
-        // chunks of independent work per thread hide the load latency)
-        uint4 v[CH][4];
+        // all of this stage's codes are loaded before any is decoded
+        uint4 v[CH][4];    // FP8: 16 codes per owned row
+        uint2 v4[CH][4];   // MXFP4: 16 codes per owned row
+        uint32_t mult[CH][4];
         for (int c = 0; c < nv; ++c) {
-          const int g = st * CH + c, h = g & 1;
+          const int g = st * CH + c, h = g % Sh::QCH;
           if (h == 0) {
             // lane 0 waits for the Q tile; the others then observe the completed
             // phase themselves (it cannot move on before this warp releases it),
@@ -342,11 +446,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0) w = tc::wait_bounded(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
             (void)tc::mbar_try_wait(qfull(qs), qph);
-          }
-          const uint8_t* q = q_base + qs * Sh::Q_BYTES + q_row + (((4 * h + c4) ^ r_lo) << 4);
+            if constexpr (WQ == WQ_MXFP4) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) v[c][i] = *reinterpret_cast<const uint4*>(q + i * 64 * Sh::QK);
-          if (h == 1 || g == nck - 1) {  // this Q tile is fully read: hand it back
+              for (int i = 0; i < 4; ++i) bs_cur[i] = bs_nxt[i];
+              if (g / Sh::QCH + 1 < nqs) load_bs(g / Sh::QCH + 1);
+            }
+          }
+          const uint8_t* qt = q_base + qs * Sh::Q_BYTES + q_row;
+          if constexpr (WQ == WQ_MXFP4) {
+            const uint8_t* q = qt + (((2 * h + (c4 >> 1)) ^ r_lo) << 4) + (c4 & 1) * 8;
+            const int blk = 2 * h + (c4 >> 1);  // block of this Q stage's row
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v4[c][i] = *reinterpret_cast<const uint2*>(q + i * 64 * Sh::Q_ROW);
+              const uint32_t wbs = blk < 4 ? bs_cur[i].x : bs_cur[i].y;
+              mult[c][i] = mx_block_multiplier((wbs >> (8 * (blk & 3))) & 0xFFu, inv_rf[i]);
+            }
+          } else {
+            const uint8_t* q = qt + (((4 * h + c4) ^ r_lo) << 4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[c][i] = *reinterpret_cast<const uint4*>(q + i * 64 * Sh::Q_ROW);
+          }
+          if (h == Sh::QCH - 1 || g == nck - 1) {  // this Q tile is fully read: hand it back
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(qempty(qs));
             if (++qs == NQ) { qs = 0; qph ^= 1u; }
@@ -360,10 +481,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t o[8];
-            e4m3x4_to_f16x4(v[c][i].x, o[0], o[1]);
-            e4m3x4_to_f16x4(v[c][i].y, o[2], o[3]);
-            e4m3x4_to_f16x4(v[c][i].z, o[4], o[5]);
-            e4m3x4_to_f16x4(v[c][i].w, o[6], o[7]);
+            if constexpr (WQ == WQ_MXFP4) {
+              mxfp4x16_to_f16x16(v4[c][i], mult[c][i], o);
+            } else {
+              e4m3x4_to_f16x4(v[c][i].x, o[0], o[1]);
+              e4m3x4_to_f16x4(v[c][i].y, o[2], o[3]);
+              e4m3x4_to_f16x4(v[c][i].z, o[4], o[5]);
+              e4m3x4_to_f16x4(v[c][i].w, o[6], o[7]);
+            }
             uint8_t* rowp = b16 + i * 8 * 1024;  // rows + 64 i
             *reinterpret_cast<uint4*>(rowp + pos0) = make_uint4(o[0], o[1], o[2], o[3]);
             *reinterpret_cast<uint4*>(rowp + pos1) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -388,6 +513,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
+      if (tc::tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, G)) continue;
       int ok = 1;
       if (lane == 0) ok = tc::wait_bounded(tfull(acc), acc_phase, abort_flag, tmo) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -453,6 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  tc::record_call_status(abort_flag, p.call_err);
   if (warp == 1) {
     __syncwarp();
     tc::tmem_dealloc(tmem_base, TMEM_COLS);
@@ -550,6 +677,92 @@ __global__ void __launch_bounds__(256) dequantize_rows_fp8_kernel(const uint8_t*
       const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
       const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
       o[j] = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-block MXFP4 quantisation of weight rows (run once, outside the forward
+// pass). For each block of 32 consecutive weights of a row: X = floor(log2
+// absmax) - 2 (0 for an all-zero block), the codes are the E2M1 values nearest
+// to w / 2^X (ties to even, saturating at +-6), two per byte with the even
+// element in the low nibble, and the block byte is X + 127 (E8M0). The row
+// factor is 2^(the largest X among the row's non-zero blocks), 1 if none.
+// One thread per block (cols / 32 per row); a block of 256 threads per row.
+// ---------------------------------------------------------------------------
+template <typename TW>
+__global__ void __launch_bounds__(256) quantize_rows_mxfp4_kernel(
+    const TW* __restrict__ w, int64_t rows, int cols, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ bscales, float* __restrict__ row_factor) {
+  constexpr int VN = Vec16<TW>::N;  // elements per 16-byte vector
+  const int nblk = cols / 32;
+  __shared__ int red[8];
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    int xmax = INT_MIN;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+      float f[32];
+      const uint4* src = reinterpret_cast<const uint4*>(w + r * cols + b * 32);
+#pragma unroll
+      for (int q = 0; q < 32 / VN; ++q) Vec16<TW>::unpack(ld_nc_v4(src + q), f + q * VN);
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      int X = 0;
+      if (amax > 0.f) {
+        int ex;
+        (void)frexpf(amax, &ex);  // amax = m 2^ex, m in [0.5, 1): floor(log2 amax) = ex - 1
+        X = ex - 3;
+        xmax = max(xmax, X);
+      }
+      uint32_t packed[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t byte = __nv_cvt_float2_to_fp4x2(
+            make_float2(ldexpf(f[2 * j], -X), ldexpf(f[2 * j + 1], -X)), __NV_E2M1,
+            cudaRoundNearest);
+        packed[j >> 2] |= (byte & 0xFFu) << (8 * (j & 3));
+      }
+      *reinterpret_cast<uint4*>(codes + r * (cols / 2) + b * 16) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      bscales[r * nblk + b] = static_cast<uint8_t>(X + 127);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) xmax = max(xmax, __shfl_xor_sync(0xffffffffu, xmax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = xmax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int m = INT_MIN;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = max(m, red[i]);
+      row_factor[r] = m == INT_MIN ? 1.0f : ldexpf(1.0f, m);
+    }
+    __syncthreads();
+  }
+}
+
+// out[r][c] = the weight an MXFP4 layer computes with, code * 2^X of its block,
+// built by the routine the GEMM converters use (fp16 code * 2^(X - X_row), then
+// the row factor 2^X_row in fp32). One thread per 16 codes.
+__global__ void __launch_bounds__(256) dequantize_rows_mxfp4_kernel(
+    const uint8_t* __restrict__ codes, const uint8_t* __restrict__ bscales,
+    const float* __restrict__ row_factor, int64_t rows, int cols, float* __restrict__ out) {
+  const int64_t vec_per_row = cols / 16;
+  const int64_t n = rows * vec_per_row;
+  const int nblk = cols / 32;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / vec_per_row;
+    const int j = (int)(i - r * vec_per_row);
+    const float rf = row_factor[r];
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + r * (cols / 2) + j * 8));
+    uint32_t o[8];
+    mxfp4x16_to_f16x16(c, mx_block_multiplier(bscales[r * nblk + j / 2], 1.0f / rf), o);
+    float4* dst = reinterpret_cast<float4*>(out + r * cols + j * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&o[2 * q]));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&o[2 * q + 1]));
+      dst[q] = make_float4(a.x * rf, a.y * rf, b.x * rf, b.y * rf);
     }
   }
 }

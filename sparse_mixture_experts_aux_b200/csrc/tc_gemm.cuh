@@ -74,7 +74,8 @@ enum { EPI_SWIGLU_TC = 0, EPI_SCALE_TC = 1 };
 struct TcGroup {
   const int32_t* tile_start;  // routed rows: [E + 1] segment starts in BM-row tiles; NULL = dense
   int E;
-  int rows;                   // dense groups: valid rows
+  int rows;                   // dense groups: valid rows; routed groups: rows of the permuted
+                              // buffers (the bounds checks of MOE_DEBUG builds)
   int n_tiles;                // output tiles per expert along N
   int k_blocks;               // K / BK
   int N;                      // output columns
@@ -93,6 +94,7 @@ struct TcParams {
   int num_groups;
   unsigned long long timeout_ns;        // limit of each pipeline wait
   unsigned long long drain_timeout_ns;  // limit of the teardown waits for work in flight
+  int* call_err;                        // the call's own status word (NULL: none)
 };
 
 struct TcMaps {
@@ -151,9 +153,10 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Same, ignoring the abort flag: used only in teardown, to let copies and
-// MMAs already in flight land before shared memory and TMEM are released.
-__device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity,
+// Same, not stopping on the abort flag (it raises it when it gives up): used
+// only in teardown, to let copies and MMAs already in flight land before
+// shared memory and TMEM are released.
+__device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                         unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t limit = wait_cycles(timeout_ns);
@@ -162,9 +165,16 @@ __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 1u && static_cast<uint64_t>(clock64() - t0) > limit) {
       atomicOr(&g_dev_error, DEVERR_TIMEOUT);
+      *abort_flag = 1;
       return false;
     }
   }
+}
+
+// After the CTA's roles have finished: a CTA that gave up anywhere records it
+// in the call's own status word as well.
+__device__ __forceinline__ void record_call_status(volatile int* abort_flag, int* call_err) {
+  if (threadIdx.x == 0 && call_err != nullptr && *abort_flag) atomicOr(call_err, DEVERR_TIMEOUT);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -321,6 +331,23 @@ __device__ __forceinline__ TileInfo decode_tile(long long tile, long long tiles0
   return ti;
 }
 
+// Builds with MOE_DEBUG: true when a tile's expert, N block or rows fall outside
+// what its tensor maps and stores cover (routed groups: the whole 128-row tile
+// inside the group's `rows` permuted rows; dense groups: its first row inside).
+// Every role of a kernel skips such a tile, so the pipeline stays in step, and
+// one producer records it in the device error word. Release builds: false.
+__device__ __forceinline__ bool tile_out_of_bounds(int e, int nb, int row0, int span,
+                                                   const TcGroup& g) {
+#if defined(MOE_DEBUG)
+  if (nb < 0 || nb >= g.n_tiles || row0 < 0) return true;
+  if (g.tile_start != nullptr) return e < 0 || e >= g.E || row0 + span > g.rows;
+  return row0 >= g.rows;
+#else
+  (void)e; (void)nb; (void)row0; (void)span; (void)g;
+  return false;
+#endif
+}
+
 // Q8: A and B are E4M3 codes (tensor maps over 16-bit elements, 2 codes each,
 // so a K step is the same 128-byte line as in bf16: 128 codes), and the
 // epilogue multiplies each accumulator by the A row's and the B column's
@@ -401,6 +428,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile(tile, tiles0, p, s_ts);
+        if (tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, p.g[ti.g])) {
+          if (me == 0) flag_bounds();
+          continue;
+        }
         const int kbs = p.g[ti.g].k_blocks;
         for (int kb = 0; kb < kbs; ++kb, ++gs) {
           if ((uint32_t)(gs & 1) != me) continue;
@@ -424,7 +455,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {  // let every copy this thread issued land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
-          if ((issued >> s) & 1u) wait_drain(full_bar(s), (last_par >> s) & 1u, drain_tmo);
+          if ((issued >> s) & 1u)
+            wait_drain(full_bar(s), (last_par >> s) & 1u, abort_flag, drain_tmo);
       }
     }
   } else if (warp == 1) {
@@ -436,6 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile(tile, tiles0, p, s_ts);
+        if (tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, p.g[ti.g])) continue;
         const int kbs = p.g[ti.g].k_blocks;
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
@@ -463,7 +496,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (acc == 0u) acc_phase ^= 1u;
       }
       tc_commit(done_bar);  // every MMA issued above has completed once this fires
-      wait_drain(done_bar, 0u, drain_tmo);
+      wait_drain(done_bar, 0u, abort_flag, drain_tmo);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -475,6 +508,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo ti = decode_tile(tile, tiles0, p, s_ts);
       const TcGroup& g = p.g[ti.g];
+      if (tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, g)) continue;
       int ok = 1;
       if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, tmo) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);  // whole warp converged and agreed
@@ -547,6 +581,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  record_call_status(abort_flag, p.call_err);
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -156,6 +156,7 @@ def routing_views(ws: torch.Tensor, x: torch.Tensor, W_g: torch.Tensor, E: int, 
         h=view(L.h, L.rows_max * d_e, x.dtype).view(L.rows_max, d_e),
         yrows=view(L.yrows, L.rows_max * d, x.dtype).view(L.rows_max, d),
         rows_max=L.rows_max, capacity=L.capacity,
+        status=view(L.status, 1, torch.int32),
         **(dict(xq=view(L.xp, L.rows_max * d, torch.uint8).view(L.rows_max, d),
                 xscale=view(L.xscale, L.rows_max, torch.float32),
                 hq=view(L.hq, L.rows_max * d_e, torch.uint8).view(L.rows_max, d_e),

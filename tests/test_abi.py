@@ -37,9 +37,19 @@ def test_library_exports_every_declared_symbol(lib):
     assert exported == set(declared_symbols())
 
 
+def test_debug_library_exports_the_same_symbols():
+    B.build(debug=True)
+    dbg = _lib.load_debug()
+    for name in declared_symbols():
+        assert hasattr(dbg, name), name
+    out = os.popen(f"nm -D --defined-only {_lib.DEBUG_LIB_PATH}").read()
+    assert set(re.findall(r"\bT (moe_\w+)", out)) == set(declared_symbols())
+
+
 def test_status_strings(lib):
     assert _lib.status_string(0) == "MOE_OK"
     assert _lib.status_string(5) == "MOE_ERR_DEVICE_TIMEOUT"
+    assert _lib.status_string(7) == "MOE_ERR_DEVICE_BOUNDS"
     assert _lib.status_string(99) == "MOE_STATUS_UNKNOWN"
 
 

@@ -6,7 +6,8 @@ context and workspace computes the right answer."""
 import pytest
 import torch
 
-from sparse_mixture_experts_aux_b200 import Workspace, _lib, forward, moe_get_device_status
+from sparse_mixture_experts_aux_b200 import (Workspace, _lib, forward, moe_get_device_status,
+                                             routing_views)
 from sparse_mixture_experts_aux_b200.inputs import Workload, make_inputs
 from tests.parity_util import compare, oracle_quantized_weights, run_gpu, run_oracle
 
@@ -32,10 +33,41 @@ def test_expired_waits_are_reported_and_the_context_survives(w):
         forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["W_shared"], k=w.k,
                 d_s=w.d_s, workspace=ws, wait_timeout_ns=1)
         torch.cuda.synchronize()
+        # the call's own status word records it, and so does the device-wide word
+        status = routing_views(ws.buf, inp["x"], inp["W_g"], w.E, w.k, 0.0, w.d_s)["status"]
+        assert int(status[0]) != 0
         assert moe_get_device_status() == _lib.MOE_ERR_DEVICE_TIMEOUT
         assert moe_get_device_status() == _lib.MOE_OK  # reading it resets it
     gpu = run_gpu(w, inp, ws)  # default limit: completes and matches the oracle
+    assert int(gpu[3]["status"][0]) == 0  # cleared by the next call
     compare(w, gpu, run_oracle(w, inp))
+
+
+def test_host_io_reports_its_own_timeout_only():
+    # two calls through the host-buffer entry point on two streams, one with
+    # waits that expire: only that call reports the timeout
+    w = Workload("timeout host io", 300, 256, 4, 320, 2, seed=46)
+    inp = make_inputs(w, device="cuda")
+    out = {}
+    for name, tmo in (("bad", 1), ("good", 0)):
+        ws = Workspace()
+        ws.get(_lib.moe_workspace_size(_lib.make_dims(w.T, w.d, w.d_e), w.E, w.k, 0.0), "cuda")
+        stream = torch.cuda.Stream()
+        dims = _lib.make_dims(w.T, w.d, w.d_e, 0, _lib.MOE_BF16, None, ws.buf, ws.buf.numel(),
+                              stream.cuda_stream, wait_timeout_ns=tmo)
+        x_host = inp["x"].cpu().pin_memory()
+        y_host = torch.empty_like(x_host).pin_memory()
+        st = _lib.moe_forward_host_io(
+            dims, x_host, torch.empty_like(inp["x"]), inp["W_r"], inp["W_g"], inp["W_u"],
+            inp["W_d"], None, w.E, w.k, 0.0, torch.empty_like(inp["x"]), y_host,
+            torch.empty(1, device="cuda"), torch.empty(1).pin_memory(),
+            torch.empty(w.E, dtype=torch.int32, device="cuda"),
+            torch.empty(w.E, dtype=torch.int32).pin_memory(), check=False)
+        out[name] = st
+    assert out == {"bad": _lib.MOE_ERR_DEVICE_TIMEOUT, "good": _lib.MOE_OK}
+    torch.cuda.synchronize()
+    assert moe_get_device_status() == _lib.MOE_ERR_DEVICE_TIMEOUT  # the device-wide word too
+    assert moe_get_device_status() == _lib.MOE_OK
 
 
 @pytest.mark.parametrize("w", [

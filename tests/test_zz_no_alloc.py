@@ -4,8 +4,10 @@ device memory for its own pool). It runs on the library's own statically
 sized scratch array instead of a caller-provided workspace.
 
 Checked here through the C ABI: its results match moe_forward's (given a
-torch-allocated workspace) on two calls in a row, and a layer that needs more
-scratch than the fixed maximum is refused before anything is enqueued. This
+torch-allocated workspace) on two calls in a row, and after calls of layers
+with another layout that leave different stale contents in the shared
+array; a layer that needs more scratch than the fixed maximum is refused
+before anything is enqueued. This
 file is collected last on purpose, so that a stop-at-first-failure run has
 already run every other test; it also passes alone in a fresh process."""
 import numpy as np
@@ -60,6 +62,46 @@ def test_no_alloc_matches_workspace_entry_point_on_two_calls(w):
         assert moe_get_device_status() == _lib.MOE_OK
         got = y.float().cpu().numpy()
         assert np.all(np.abs(got - ref) <= tol * np.maximum(1.0, np.abs(ref)))
+        assert torch.equal(counts.cpu(), counts_ref.cpu())
+        assert float(aux.cpu()[0]) == pytest.approx(float(aux_ref.cpu()[0]), rel=1e-6)
+
+
+def _no_alloc_call(w, inp):
+    stream = torch.cuda.current_stream().cuda_stream
+    dt = _lib.MOE_BF16 if w.dtype == "bf16" else _lib.MOE_F32
+    dims = _lib.make_dims(w.T, w.d, w.d_e, w.d_s, dt, inp["router_bias"], None, 0, stream)
+    y = torch.full_like(inp["x"], float("nan"))
+    aux = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
+    counts = torch.full((w.E,), -1, dtype=torch.int32, device="cuda")
+    st = _lib.moe_forward_no_alloc(dims, inp["x"], inp["W_r"], inp["W_g"], inp["W_u"],
+                                   inp["W_d"], inp["W_shared"], w.E, w.k, w.capacity_factor,
+                                   y, aux, counts, check=False)
+    assert st == _lib.MOE_OK, _lib.status_string(st)
+    torch.cuda.synchronize()
+    assert moe_get_device_status() == _lib.MOE_OK
+    return y, aux, counts
+
+
+def test_no_alloc_after_a_different_layout():
+    # Every call shares the scratch array and finds what the previous call left:
+    # here each call follows a layer with another E, capacity cut, shared expert
+    # and row layout, so stale segment starts, row gates, logits splits and rows
+    # of the other layout sit in the array when it starts.
+    layers = [CASES[1], MIXTRAL_DECODE, CASES[1], MIXTRAL_DECODE]
+    inputs = {w.name: make_inputs(w, device="cuda") for w in layers[:2]}
+    refs = {}
+    for w in layers[:2]:
+        inp = inputs[w.name]
+        refs[w.name] = forward(inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"],
+                               inp["W_shared"], k=w.k, capacity_factor=w.capacity_factor,
+                               router_bias=inp["router_bias"], d_s=w.d_s, workspace=Workspace())
+    torch.cuda.synchronize()
+    for w in layers:
+        y, aux, counts = _no_alloc_call(w, inputs[w.name])
+        y_ref, aux_ref, counts_ref = refs[w.name]
+        ref = y_ref.float().cpu().numpy()
+        got = y.float().cpu().numpy()
+        assert np.all(np.abs(got - ref) <= Y_TOL[w.dtype] * np.maximum(1.0, np.abs(ref))), w.name
         assert torch.equal(counts.cpu(), counts_ref.cpu())
         assert float(aux.cpu()[0]) == pytest.approx(float(aux_ref.cpu()[0]), rel=1e-6)
 
