@@ -51,11 +51,13 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral",
                     choices=["mixtral", "deepseek_v3", "switch_zipf", "decode", "tiny_fp32",
-                             "mixtral_profile", "decode_profile", "routing_profile"])
-    ap.add_argument("--weights", choices=["dtype", "fp8", "w8a8"], default="dtype",
+                             "mixtral_profile", "decode_profile", "routing_profile",
+                             "dsv3_routing_profile"])
+    ap.add_argument("--weights", choices=["dtype", "fp8", "w8a8", "mxfp4"], default="dtype",
                     help="expert weights in the activation dtype; E4M3 codes with per-row "
-                         "scales (quantised once by the library before timing); or those and "
-                         "E4M3 activations inside the experts (W8A8)")
+                         "scales (quantised once by the library before timing); those and "
+                         "E4M3 activations inside the experts (W8A8); or MXFP4 codes with "
+                         "per-32 block scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
@@ -69,7 +71,8 @@ def workload_by_name(name):
     return {"mixtral": I.MIXTRAL, "deepseek_v3": I.DEEPSEEK_V3, "switch_zipf": I.SWITCH_ZIPF,
             "decode": I.MIXTRAL_DECODE, "tiny_fp32": I.TINY_F32,
             "mixtral_profile": I.MIXTRAL_PROFILE, "decode_profile": I.DECODE_PROFILE,
-            "routing_profile": I.ROUTING_PROFILE}[name]
+            "routing_profile": I.ROUTING_PROFILE,
+            "dsv3_routing_profile": I.DSV3_ROUTING_PROFILE}[name]
 
 
 def load_peaks():
@@ -223,11 +226,14 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------------------- our arm
-def step_work(w, counts, fp8: bool):
+def step_work(w, counts, weights: str = "dtype"):
     """Algorithmic work of one step from its own routing counts: kept
     assignments, touched experts, FLOPs of the two GEMMs, and the bytes each
     GEMM and the whole layer must move at least (touched expert weights once,
-    plus the rows a GEMM reads and writes; x in and y out for the layer)."""
+    plus the rows a GEMM reads and writes; x in and y out for the layer).
+    weights: "dtype", "fp8", "w8a8" (one byte per weight, 4 per weight row) or
+    "mxfp4" (half a byte per weight, one per 32, 4 per weight row)."""
+    fp8 = weights != "dtype"
     from sparse_mixture_experts_aux_b200 import _lib
     C = _lib.moe_capacity(w.T, w.E, w.k, w.capacity_factor)
     C = None if C < 0 else C
@@ -235,7 +241,8 @@ def step_work(w, counts, fp8: bool):
     kept = sum(kept_e)
     touched = sum(1 for c in kept_e if c > 0)
     esz = 2 if w.dtype == "bf16" else 4
-    wsz = 1 if fp8 else esz  # bytes per expert weight (+ 4 per row of scales with FP8)
+    # bytes per expert weight (+ 4 per weight row of scales when quantised)
+    wsz = (0.5 + 1.0 / 32) if weights == "mxfp4" else (1 if fp8 else esz)
     sh = w.T if w.d_s else 0
     flops_up = 2 * kept * w.d * 2 * w.d_e + 2 * sh * w.d * 2 * w.d_s
     flops_down = 2 * kept * w.d_e * w.d + 2 * sh * w.d_s * w.d
@@ -248,6 +255,13 @@ def step_work(w, counts, fp8: bool):
     return dict(C=C, kept=kept, touched=touched, flops_up=flops_up, flops_down=flops_down,
                 flops=flops_up + flops_down, bytes_up=bytes_up, bytes_down=bytes_down,
                 w_bytes=w_bytes, act_bytes=2 * w.T * w.d * esz)
+
+
+def launches_per_step(w, act_fp8: bool) -> int:
+    """Kernels one forward call enqueues: the 7 steps, with the bf16 router step
+    as two kernels (weight split + tensor-core logits) and, with E4M3
+    activations, the x and H quantisers."""
+    return 7 + (1 if w.dtype == "bf16" else 0) + (2 if act_fp8 else 0)
 
 
 def kernel_roofline(flops, nbytes, ms, tensor_peak, hbm_peak):
@@ -286,7 +300,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
     from sparse_mixture_experts_aux_b200 import (KERNEL_NAMES, MOE_NUM_KERNELS, Workspace,
                                                  forward, _lib, moe_get_device_status,
-                                                 quantize_fp8)
+                                                 quantize_fp8, quantize_mxfp4)
     from sparse_mixture_experts_aux_b200.events import KernelEvents
     from sparse_mixture_experts_aux_b200.inputs import MIXTRAL_DECODE, make_inputs, make_x
     from oracle import moe_oracle as O  # cpu_baseline leg only
@@ -302,10 +316,18 @@ def run_ours(args, rank, world, local_rank):
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     counts = torch.empty(w.E, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    fp8 = args.weights in ("fp8", "w8a8")
+    fp8 = args.weights in ("fp8", "w8a8", "mxfp4")
     act_fp8 = args.weights == "w8a8"
-    scales = None
-    if fp8:  # one-off weight preparation, untimed
+    scales = bscales = None
+    if args.weights == "mxfp4":  # one-off weight preparation, untimed
+        parts, bparts = [], []
+        for name in ("W_g", "W_u", "W_d"):
+            inp[name], bs, rf = quantize_mxfp4(inp[name])
+            parts.append(rf.reshape(-1))
+            bparts.append(bs.reshape(-1))
+        scales, bscales = torch.cat(parts), torch.cat(bparts)
+        torch.cuda.synchronize()
+    elif fp8:
         parts = []
         for name in ("W_g", "W_u", "W_d"):
             inp[name], sc = quantize_fp8(inp[name])
@@ -318,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
                 inp["W_shared"], k=w.k, capacity_factor=w.capacity_factor,
                 router_bias=inp["router_bias"], d_s=w.d_s, workspace=ws, stream=stream,
                 events=events, y=yb, aux=aux, counts=counts, weight_scales=scales,
-                act_fp8=act_fp8)
+                act_fp8=act_fp8, weight_block_scales=bscales)
 
     def barrier():
         if world > 1:
@@ -344,7 +366,7 @@ def run_ours(args, rank, world, local_rank):
         kv.close()
     ms_max = max_over_ranks(ms, dev)
 
-    wk = step_work(w, counts.cpu().numpy().astype("int64"), fp8)
+    wk = step_work(w, counts.cpu().numpy().astype("int64"), args.weights)
     peaks, peaks_src = load_peaks()
     # Headline tensor peak: the burst cuBLAS figure (a kernel timed in a short run at
     # full clock, as this one is); the sustained, power-capped figure is reported
@@ -388,7 +410,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": dict(config_of(w, "inputs larger than L2: %.2f GB of expert weights streamed "
                                     "per step; x rotates over %d batches" % (wk["w_bytes"] / 1e9, R)),
-                       weights="e4m3 codes + fp32 row scales" if fp8 else w.dtype,
+                       weights=("e2m1 codes + e8m0 block scales (32) + fp32 row factors"
+                                if args.weights == "mxfp4" else
+                                "e4m3 codes + fp32 row scales" if fp8 else w.dtype),
                        activations="e4m3 rows + fp32 row scales in the experts" if act_fp8
                        else w.dtype),
         "roofline": rl,
@@ -401,8 +425,7 @@ def run_ours(args, rank, world, local_rank):
                   "dropped_fraction": O.dropped_fraction(counts.cpu().numpy(), wk["C"], w.T, w.k),
                   "aux": float(aux.cpu()[0])},
         "kernel_ms": {KERNEL_NAMES[j]: per_kernel[j] for j in range(MOE_NUM_KERNELS)},
-        # W8A8 adds the x and H quantisers to the 7 kernels of a step
-        "gpu_launches": (MOE_NUM_KERNELS + (2 if act_fp8 else 0)) * args.steps * world,
+        "gpu_launches": launches_per_step(w, act_fp8) * args.steps * world,
         "clocks": clk,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
     }
@@ -420,6 +443,7 @@ def run_ours(args, rank, world, local_rank):
         x_host = [xs[j].cpu().pin_memory() for j in range(2)]
         nbytes = ws.buf.numel()
         fmt = (_lib.MOE_WEIGHTS_FP8_W8A8 if act_fp8 else
+               _lib.MOE_WEIGHTS_MXFP4 if args.weights == "mxfp4" else
                _lib.MOE_WEIGHTS_FP8 if fp8 else _lib.MOE_WEIGHTS_DTYPE)
         bufs = []
         for sidx in range(NSTR):
@@ -433,7 +457,8 @@ def run_ours(args, rank, world, local_rank):
             b["dims"] = _lib.make_dims(w.T, w.d, w.d_e, w.d_s,
                                        _lib.MOE_BF16 if w.dtype == "bf16" else _lib.MOE_F32,
                                        inp["router_bias"], wsb, nbytes, streams[sidx].cuda_stream,
-                                       weight_format=fmt, weight_scales=scales)
+                                       weight_format=fmt, weight_scales=scales,
+                                       weight_block_scales=bscales)
             bufs.append(b)
 
         def e2e_run(sidx, first, count):
@@ -487,7 +512,7 @@ def run_ours(args, rank, world, local_rank):
         def dcall(i, events=None):
             forward(xl[i], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], None, k=wd.k,
                     workspace=ws, stream=stream, events=events, y=yd, aux=aux, counts=cd,
-                    weight_scales=scales, act_fp8=act_fp8)
+                    weight_scales=scales, act_fp8=act_fp8, weight_block_scales=bscales)
 
         for i in range(max(3, args.warmup)):
             dcall(i)
@@ -503,7 +528,7 @@ def run_ours(args, rank, world, local_rank):
         for kv in dkev:
             kv.close()
         dms_max = max_over_ranks(dms, dev)
-        dwk = step_work(wd, cd.cpu().numpy().astype("int64"), fp8)
+        dwk = step_work(wd, cd.cpu().numpy().astype("int64"), args.weights)
         d_ms = dms_max / n
         d_roof = max(dwk["flops"] / (tensor_peak * 1e12),
                      (dwk["w_bytes"] + dwk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
@@ -520,7 +545,7 @@ def run_ours(args, rank, world, local_rank):
                      **kernel_roofline(dwk["flops_down"], dwk["bytes_down"], dk[5], tensor_peak,
                                        hbm_peak)},
             "kernel_ms": {KERNEL_NAMES[j]: dk[j] for j in range(MOE_NUM_KERNELS)},
-            "gpu_launches": (MOE_NUM_KERNELS + (2 if act_fp8 else 0)) * n * world,
+            "gpu_launches": launches_per_step(wd, act_fp8) * n * world,
             "clocks": dclk,
             "l2": "weights (%.2f GB) larger than L2; each call reads its own x" % (dwk["w_bytes"] / 1e9),
         }

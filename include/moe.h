@@ -75,16 +75,20 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
-/* Number of kernels moe_forward enqueues, in order: router logits, routing
+/* Number of steps moe_forward enqueues, in order: router logits, routing
  * (softmax / top-k / gates / ranks), scan (counts, capacity, offsets, aux),
  * scatter (permute x rows), gate/up grouped GEMM + SwiGLU, down grouped GEMM
- * + gate scaling, combine (un-permute + shared expert). */
+ * + gate scaling, combine (un-permute + shared expert). Each step is one
+ * kernel, except the router step with bf16 x (two: the exact bf16 split of W_r
+ * and the tensor-core logits) and, with MOE_WEIGHTS_FP8_W8A8, the scatter and
+ * down steps (each one more: the x and H quantisers). */
 #define MOE_NUM_KERNELS 7
 
 /* Limits of this library: 1 <= k <= 32, k <= E <= 1024; bf16 needs d, d_e, d_s
  * multiples of 64; fp32 needs them multiples of 32; T < 2^31 / max(k, 1);
- * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group; the FP8
- * weight formats need bf16 x and no shared expert (d_s = 0). */
+ * n_group <= 32 and a divisor of E, k <= topk_group * E / n_group; the
+ * quantised weight formats need bf16 x and no shared expert (d_s = 0), and
+ * MXFP4 needs d and d_e multiples of 256. */
 
 /*
  * Routing variants (gate_mode, selection_bias, n_group / topk_group).
@@ -132,13 +136,38 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * FP8 on both GEMM operands (W8A8): the weights as for MOE_WEIGHTS_FP8, and
  * the routed experts' inputs quantised the same way, one fp32 scale per row:
  * each token row of x (absmax over d) and each routed hidden row H (absmax
- * over d_e, after H is rounded to bf16) becomes E4M3 codes * scale. The expert
+ * over d_e, from H's fp32 value) becomes E4M3 codes * scale. The expert
  * GEMMs then run E4M3 x E4M3 -> fp32 on the tensor cores, and both scales
  * multiply the accumulator. This
  * changes the numbers (activations carry 3 mantissa bits): it is a different
  * layer from MOE_WEIGHTS_FP8, not a faster route to the same one.
  */
 #define MOE_WEIGHTS_FP8_W8A8 2
+/*
+ * MXFP4 expert weights (weight-only; the 4-bit format gpt-oss quantises its
+ * experts to: AI Engineering Illustrated "Mixture of Experts", "Trade-offs to
+ * weigh"). The pages give no format details; this library follows the Open
+ * Compute microscaling convention. Each block of 32 consecutive weights of a
+ * row (along K) shares X = floor(log2(absmax of the block)) - 2 (X = 0 for an
+ * all-zero block); each weight becomes the E2M1 value (magnitudes 0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6) nearest to w / 2^X, ties to the even mantissa, saturating
+ * at +-6; the layer computes with code * 2^X. Storage, per weight stack:
+ *   codes        uint8 [rows, K / 2]: two codes per byte, the even-K element in
+ *                the low nibble (bit 3 = sign, bits 2..1 = exponent, bit 0 =
+ *                mantissa); passed as W_g, W_u, W_d;
+ *   block scales uint8 [rows, K / 32]: X + 127 (E8M0); the three stacks' one
+ *                after another form moe_dims.weight_block_scales;
+ *   row factors  fp32 [rows]: 2^(the largest X among the row's non-zero blocks),
+ *                1 for an all-zero row; the three stacks' one after another form
+ *                moe_dims.weight_scales.
+ * moe_quantize_mxfp4 writes all three. The GEMMs stream the codes, decode them
+ * on chip to fp16 (the E2M1 value times 2^(X - X_row), exact while
+ * X >= X_row - 23; weights of smaller blocks are rounded to multiples of
+ * 2^(X_row - 24)) and apply the row factor to the fp32 accumulator. As with
+ * FP8 weight-only, the routed activations and H are held in fp16 on this path.
+ * Needs bf16 x, no shared expert, and d, d_e multiples of 256.
+ */
+#define MOE_WEIGHTS_MXFP4 3
 
 typedef struct {
   int64_t T;                 /* tokens in this call (0 allowed: empty batch) */
@@ -168,16 +197,24 @@ typedef struct {
                                 MOE_WEIGHTS_FP8 (1): E4M3 codes (uint8) with per-row scales,
                                 see moe_quantize_fp8 (bf16 activations, no shared expert);
                                 MOE_WEIGHTS_FP8_W8A8 (2): the same weights, and E4M3
-                                activations inside the experts (see above) */
-  const float* weight_scales; /* MOE_WEIGHTS_FP8: device fp32, the per-row scales of the three
-                                 stacks one after another: W_g [E*d_e], W_u [E*d_e],
-                                 W_d [E*d] (what moe_quantize_fp8 writes for each stack) */
+                                activations inside the experts (see above);
+                                MOE_WEIGHTS_MXFP4 (3): packed E2M1 codes with block scales
+                                and row factors, see above and moe_quantize_mxfp4 */
+  const float* weight_scales; /* MOE_WEIGHTS_FP8(_W8A8): device fp32, the per-row scales of the
+                                 three stacks one after another: W_g [E*d_e], W_u [E*d_e],
+                                 W_d [E*d] (what moe_quantize_fp8 writes for each stack);
+                                 MOE_WEIGHTS_MXFP4: the row factors, in the same order */
   uint64_t wait_timeout_ns;  /* limit of each device-side mbarrier wait in the GEMM
                                 kernels; 0 = default (4 s). A tiny value makes the waits
                                 expire on purpose: the kernels then record
                                 MOE_ERR_DEVICE_TIMEOUT, let their in-flight copies and
                                 MMAs land, free TMEM and return (outputs undefined), and
                                 the context stays usable. */
+  const uint8_t* weight_block_scales; /* MOE_WEIGHTS_MXFP4 only: device uint8 E8M0 block
+                                 scales, 16-byte aligned, of the three stacks one after
+                                 another: W_g [E*d_e*(d/32)], W_u [E*d_e*(d/32)],
+                                 W_d [E*d*(d_e/32)] (what moe_quantize_mxfp4 writes);
+                                 ignored otherwise */
 } moe_dims;
 
 /* Bytes of device workspace moe_forward needs for this layer (0 on invalid
@@ -243,7 +280,8 @@ typedef struct {
   size_t tile_start;  /* int32 [E + 1]  first 128-row tile of each expert's
                                         segment; [E] = number of routed tiles */
   size_t xp;          /* dtype [rows_max, d]   x rows grouped by expert */
-  size_t h;           /* dtype [rows_max, d_e] SwiGLU hidden rows */
+  size_t h;           /* dtype [rows_max, d_e] SwiGLU hidden rows (fp32 with
+                         MOE_WEIGHTS_FP8_W8A8; fp16 with the other quantised formats) */
   size_t yrows;       /* dtype [rows_max, d]   gate-scaled expert outputs */
   int64_t rows_max;   /* rows reserved for the permuted buffers */
   int64_t capacity;   /* C, or -1 */
@@ -299,6 +337,34 @@ MOE_API moe_status moe_quantize_fp8(const void* w, int32_t dtype, int64_t rows, 
  */
 MOE_API moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales, int64_t rows,
                                       int32_t cols, float* out, void* stream);
+
+/*
+ * MXFP4 quantisation of `rows` rows of `cols` weights (device, `dtype` =
+ * MOE_BF16 or MOE_F32, row-major; cols a multiple of 32) with the rule above,
+ * asynchronously on `stream`: codes (device uint8 [rows, cols / 2], 16-byte
+ * aligned), block scales (device uint8 [rows, cols / 32]) and row factors
+ * (device fp32 [rows]). For a routed expert stack, W_g [E, d_e, d] is
+ * rows = E * d_e, cols = d (likewise W_u), and W_d [E, d, d_e] is rows = E * d,
+ * cols = d_e. Returns MOE_ERR_INVALID_ARG for null pointers, rows < 0, cols not
+ * a multiple of 32, a bad dtype, or w / codes not 16-byte aligned (nothing is
+ * launched), MOE_ERR_CUDA on launch failure.
+ */
+MOE_API moe_status moe_quantize_mxfp4(const void* w, int32_t dtype, int64_t rows, int32_t cols,
+                                      uint8_t* codes, uint8_t* block_scales, float* row_factors,
+                                      void* stream);
+
+/*
+ * The weights an MXFP4 layer computes with: out[r][c] = value(code) * 2^X of
+ * its block (device fp32 [rows, cols]), built by the routine the GEMM kernels
+ * use (fp16 code * 2^(X - X_row), then times the row factor in fp32), so it is
+ * exact under the same condition. For checking a quantised stack or
+ * materialising it. Returns MOE_ERR_INVALID_ARG for null pointers, rows < 0,
+ * cols not a multiple of 32, or codes / out not 16-byte aligned (nothing is
+ * launched), MOE_ERR_CUDA on launch failure.
+ */
+MOE_API moe_status moe_dequantize_mxfp4(const uint8_t* codes, const uint8_t* block_scales,
+                                        const float* row_factors, int64_t rows, int32_t cols,
+                                        float* out, void* stream);
 
 /*
  * moe_forward for callers that cannot allocate device memory. The pages have

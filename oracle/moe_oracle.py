@@ -46,7 +46,6 @@ import math
 from typing import Callable, Optional, Sequence
 
 import numpy as np
-import torch
 
 __all__ = [
     "router_logits", "softmax_all", "top_k", "gates_softmax_topk", "gates_renormalised",
@@ -54,7 +53,7 @@ __all__ = [
     "GATE_RENORM", "GATE_RAW", "GATE_SIGMOID", "sigmoid_affinity", "balance_probs",
     "selection_scores", "group_eligible", "select_experts", "gates_for_mode",
     "E4M3_MAX", "e4m3_round", "e4m3_encode", "e4m3_decode", "quantize_rows_fp8",
-    "dequantize_rows_fp8", "fake_quant_rows_fp8", "round_bf16", "swiglu_ffn_w8a8",
+    "dequantize_rows_fp8", "fake_quant_rows_fp8", "swiglu_ffn_w8a8",
     "E2M1_MAX", "MX_BLOCK", "e2m1_round", "e2m1_encode", "e2m1_decode", "quantize_rows_mxfp4",
     "dequantize_rows_mxfp4",
     "aux_statistic", "aux_statistic_top1", "dropped_fraction", "moe_forward",
@@ -517,12 +516,6 @@ def fake_quant_rows_fp8(a) -> np.ndarray:
     """Rows of `a` through the per-row E4M3 quantiser and back (fp64, exact)."""
     codes, scales = quantize_rows_fp8(a)
     return dequantize_rows_fp8(codes, scales)
-
-
-def round_bf16(a) -> np.ndarray:
-    """fp64 -> fp32 -> bf16, each step round-to-nearest-even (torch's casts), as fp64."""
-    t = torch.tensor(np.asarray(a, dtype=np.float64), dtype=torch.float32)
-    return t.to(torch.bfloat16).to(torch.float64).numpy()
 
 
 def swiglu_ffn_w8a8(x, W_g, W_u, W_d) -> np.ndarray:

@@ -25,13 +25,14 @@ MOE_NO_ALLOC_WORKSPACE_BYTES = 64 << 20
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_GATE_RENORM, MOE_GATE_RAW, MOE_GATE_SIGMOID = 0, 1, 2
-MOE_WEIGHTS_DTYPE, MOE_WEIGHTS_FP8, MOE_WEIGHTS_FP8_W8A8 = 0, 1, 2
+MOE_WEIGHTS_DTYPE, MOE_WEIGHTS_FP8, MOE_WEIGHTS_FP8_W8A8, MOE_WEIGHTS_MXFP4 = 0, 1, 2, 3
 MOE_NUM_KERNELS = 7
 KERNEL_NAMES = ("router_logits", "route", "scan", "scatter", "gate_up_swiglu", "down_scale", "combine")
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_forward", "moe_forward_host_io",
             "moe_workspace_layout", "moe_get_device_status", "moe_status_string",
-            "moe_forward_no_alloc", "moe_quantize_fp8", "moe_dequantize_fp8")
+            "moe_forward_no_alloc", "moe_quantize_fp8", "moe_dequantize_fp8",
+            "moe_quantize_mxfp4", "moe_dequantize_mxfp4")
 
 
 class moe_dims(ctypes.Structure):
@@ -53,6 +54,7 @@ class moe_dims(ctypes.Structure):
         ("weight_format", ctypes.c_int32),
         ("weight_scales", ctypes.c_void_p),
         ("wait_timeout_ns", ctypes.c_uint64),
+        ("weight_block_scales", ctypes.c_void_p),
     ]
 
 
@@ -131,6 +133,10 @@ def _open(path: str) -> ctypes.CDLL:
     lib.moe_quantize_fp8.restype = i32
     lib.moe_dequantize_fp8.argtypes = [vp, vp, ctypes.c_int64, i32, vp, vp]
     lib.moe_dequantize_fp8.restype = i32
+    lib.moe_quantize_mxfp4.argtypes = [vp, i32, ctypes.c_int64, i32, vp, vp, vp, vp]
+    lib.moe_quantize_mxfp4.restype = i32
+    lib.moe_dequantize_mxfp4.argtypes = [vp, vp, vp, ctypes.c_int64, i32, vp, vp]
+    lib.moe_dequantize_mxfp4.restype = i32
     return lib
 
 
@@ -154,7 +160,7 @@ def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, rou
               workspace=None, workspace_bytes: int = 0, stream: int = 0, events=None,
               gate_mode: int = 0, wait_timeout_ns: int = 0, selection_bias=None,
               n_group: int = 0, topk_group: int = 0, weight_format: int = MOE_WEIGHTS_DTYPE,
-              weight_scales=None) -> moe_dims:
+              weight_scales=None, weight_block_scales=None) -> moe_dims:
     """Fill a moe_dims. `events` is a ctypes array of cudaEvent_t handles or None."""
     dims = moe_dims()
     dims.T, dims.d, dims.d_e, dims.d_s = int(T), int(d), int(d_e), int(d_s)
@@ -169,6 +175,7 @@ def make_dims(T: int, d: int, d_e: int, d_s: int = 0, dtype: int = MOE_BF16, rou
     dims.n_group, dims.topk_group = int(n_group), int(topk_group)
     dims.weight_format = int(weight_format)
     dims.weight_scales = _ptr(weight_scales) or None
+    dims.weight_block_scales = _ptr(weight_block_scales) or None
     return dims
 
 
@@ -235,3 +242,19 @@ def moe_dequantize_fp8(codes, scales, rows: int, cols: int, out, stream: int = 0
     """Raw call: returns the status code."""
     return int(load().moe_dequantize_fp8(_ptr(codes) or None, _ptr(scales) or None, int(rows),
                                          int(cols), _ptr(out) or None, int(stream) or None))
+
+
+def moe_quantize_mxfp4(w, dtype: int, rows: int, cols: int, codes, block_scales, row_factors,
+                       stream: int = 0) -> int:
+    """Raw call: returns the status code."""
+    return int(load().moe_quantize_mxfp4(_ptr(w) or None, int(dtype), int(rows), int(cols),
+                                         _ptr(codes) or None, _ptr(block_scales) or None,
+                                         _ptr(row_factors) or None, int(stream) or None))
+
+
+def moe_dequantize_mxfp4(codes, block_scales, row_factors, rows: int, cols: int, out,
+                         stream: int = 0) -> int:
+    """Raw call: returns the status code."""
+    return int(load().moe_dequantize_mxfp4(_ptr(codes) or None, _ptr(block_scales) or None,
+                                           _ptr(row_factors) or None, int(rows), int(cols),
+                                           _ptr(out) or None, int(stream) or None))

@@ -14,6 +14,7 @@
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
 #include "tc_f8_gemm.cuh"
+#include "router_tc.cuh"
 
 namespace {
 
@@ -35,9 +36,11 @@ struct Plan {
   int nblk;   // routing chunks
   int router_split;    // K chunks of the router product
   bool router_narrow;  // few experts, many tokens: warp-per-token-group router kernel
+  bool router_tc;      // bf16 x: split-precision tensor-core router
+  int router_n;        // tensor-core router: experts per tile
   int64_t rows_max;
   size_t o_logits, o_idx, o_gate, o_lrank, o_slot, o_hist, o_base, o_psum_part, o_probsum,
-      o_tile_start, o_pair_start, o_status, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys,
+      o_tile_start, o_pair_start, o_status, o_wsplit, o_rowgate, o_xp, o_h, o_yrows, o_hs, o_ys,
       // E4M3 activations (MOE_WEIGHTS_FP8_W8A8): x codes and scales per token,
       // scales of the permuted x rows, H codes and scales per permuted row
       o_xq, o_sx, o_xsc, o_hq, o_hsc, total;
@@ -72,13 +75,36 @@ moe_status check_dims(const moe_dims* dims, int E, int k, float cf) {
       dims->T * static_cast<int64_t>(E) >= (int64_t(1) << 40))
     return MOE_ERR_UNSUPPORTED;
   if (dims->weight_format != MOE_WEIGHTS_DTYPE && dims->weight_format != MOE_WEIGHTS_FP8 &&
-      dims->weight_format != MOE_WEIGHTS_FP8_W8A8)
+      dims->weight_format != MOE_WEIGHTS_FP8_W8A8 && dims->weight_format != MOE_WEIGHTS_MXFP4)
     return MOE_ERR_INVALID_ARG;
   if (dims->weight_format != MOE_WEIGHTS_DTYPE && (dims->dtype != MOE_BF16 || dims->d_s != 0))
+    return MOE_ERR_UNSUPPORTED;
+  // MXFP4: whole 256-deep code stages (eight 32-weight blocks) along both K extents
+  if (dims->weight_format == MOE_WEIGHTS_MXFP4 && (dims->d % 256 || dims->d_e % 256))
     return MOE_ERR_UNSUPPORTED;
   const int mult = dims->dtype == MOE_BF16 ? 64 : 32;
   if (dims->d % mult || dims->d_e % mult || dims->d_s % mult) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
+}
+
+// Tensor-core router: experts per tile (E rounded up to the MMA's multiple of
+// 16, at most 128).
+int router_tc_n(int E) {
+  const int n = (E + 15) / 16 * 16;
+  return n < moe::rtc::MAX_N ? n : moe::rtc::MAX_N;
+}
+
+// Tensor-core router: K splits so that the tiles about fill the 148 SMs of a
+// B200 (at most 16, whole 64-deep blocks, at least 8 blocks each). Depends only
+// on the shape, so the workspace size does too.
+int router_tc_split_k(int64_t T, int E, int d) {
+  const int64_t tiles = ((T + moe::rtc::BM - 1) / moe::rtc::BM) *
+                        ((E + router_tc_n(E) - 1) / router_tc_n(E));
+  const int kb = d / moe::rtc::BK;
+  int split = 1;
+  while (split < 16 && tiles * split * 2 <= 148 && kb % (2 * split) == 0 && kb / (2 * split) >= 8)
+    split *= 2;
+  return split;
 }
 
 Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
@@ -102,9 +128,15 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
     return o;
   };
   const size_t T = static_cast<size_t>(p.T), TK = T * k, R = static_cast<size_t>(p.rows_max);
-  p.router_narrow = E <= 16;
-  p.router_split = p.router_narrow ? moe::narrow_split_k(p.T, E, p.d)
-                                   : moe::router_wide_split_k(p.T, E, p.d);
+  p.router_tc = p.bf16;
+  p.router_narrow = !p.router_tc && E <= 16;
+  if (p.router_tc) {
+    p.router_n = router_tc_n(E);
+    p.router_split = router_tc_split_k(p.T, E, p.d);
+  } else {
+    p.router_split = p.router_narrow ? moe::narrow_split_k(p.T, E, p.d)
+                                     : moe::router_wide_split_k(p.T, E, p.d);
+  }
   p.o_logits = take(static_cast<size_t>(p.router_split) * T * E * 4);
   p.o_idx = take(TK * 4);
   p.o_gate = take(TK * 4);
@@ -117,9 +149,12 @@ Plan make_plan(const moe_dims* dims, int E, int k, float cf) {
   p.o_tile_start = take(static_cast<size_t>(E + 1) * 4);
   p.o_pair_start = take(static_cast<size_t>(E + 1) * 4);
   p.o_status = take(4);  // the call's own device status word
+  // tensor-core router: the hi / mid / lo bf16 terms of W_r, [3][E][d]
+  p.o_wsplit = take(p.router_tc ? static_cast<size_t>(3) * E * p.d * 2 : 0);
   p.o_rowgate = take(R * 4);
   p.o_xp = take(R * p.d * p.esz);
-  p.o_h = take(R * p.de * p.esz);
+  // H: fp32 with E4M3 activations (quantised per row from its fp32 value)
+  p.o_h = take(R * p.de * (dims->weight_format == MOE_WEIGHTS_FP8_W8A8 ? 4 : p.esz));
   p.o_yrows = take(R * p.d * p.esz);
   p.o_hs = take(p.ds ? T * p.ds * p.esz : 0);
   p.o_ys = take(p.ds ? T * p.d * p.esz : 0);
@@ -158,24 +193,37 @@ bool tc_attr() {
                               moe::tc::TcShape<AR>::SMEM_BYTES) == cudaSuccess;
 }
 
-template <int EPI, int AR>
+template <int EPI, int AR, int WQ>
 bool f8_attr() {
-  return cudaFuncSetAttribute(moe::tcf8::tc_f8_grouped_gemm_kernel<EPI, AR>,
+  return cudaFuncSetAttribute(moe::tcf8::tc_f8_grouped_gemm_kernel<EPI, AR, WQ>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              moe::tcf8::F8Shape<AR>::SMEM_BYTES) == cudaSuccess;
+                              moe::tcf8::F8Shape<AR, WQ>::SMEM_BYTES) == cudaSuccess;
 }
 
-template <int EPI>
+template <int WQ>
+bool f8_attrs() {
+  using moe::tc::EPI_SWIGLU_TC;
+  using moe::tc::EPI_SCALE_TC;
+  return f8_attr<EPI_SWIGLU_TC, 128, WQ>() && f8_attr<EPI_SCALE_TC, 128, WQ>() &&
+         f8_attr<EPI_SWIGLU_TC, 64, WQ>() && f8_attr<EPI_SCALE_TC, 64, WQ>() &&
+         f8_attr<EPI_SWIGLU_TC, 32, WQ>() && f8_attr<EPI_SCALE_TC, 32, WQ>();
+}
+
+// Quantised-weight grouped GEMM (WQ: FP8 or MXFP4 codes) with an activation box
+// of `ar` rows.
+template <int EPI, int WQ>
 void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
                const moe::tcf8::F8Params& fp) {
   using namespace moe::tcf8;
   if (ar == 32)
-    tc_f8_grouped_gemm_kernel<EPI, 32><<<grid, NUM_THREADS, F8Shape<32>::SMEM_BYTES, st>>>(maps, fp);
+    tc_f8_grouped_gemm_kernel<EPI, 32, WQ>
+        <<<grid, NUM_THREADS, F8Shape<32, WQ>::SMEM_BYTES, st>>>(maps, fp);
   else if (ar == 64)
-    tc_f8_grouped_gemm_kernel<EPI, 64><<<grid, NUM_THREADS, F8Shape<64>::SMEM_BYTES, st>>>(maps, fp);
+    tc_f8_grouped_gemm_kernel<EPI, 64, WQ>
+        <<<grid, NUM_THREADS, F8Shape<64, WQ>::SMEM_BYTES, st>>>(maps, fp);
   else
-    tc_f8_grouped_gemm_kernel<EPI, 128>
-        <<<grid, NUM_THREADS, F8Shape<128>::SMEM_BYTES, st>>>(maps, fp);
+    tc_f8_grouped_gemm_kernel<EPI, 128, WQ>
+        <<<grid, NUM_THREADS, F8Shape<128, WQ>::SMEM_BYTES, st>>>(maps, fp);
 }
 
 // 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32);
@@ -251,12 +299,12 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 64, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64, true>() ||
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 32, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32, true>())
       return MOE_ERR_CUDA;
-    if (!f8_attr<moe::tc::EPI_SWIGLU_TC, 128>() || !f8_attr<moe::tc::EPI_SCALE_TC, 128>() ||
-        !f8_attr<moe::tc::EPI_SWIGLU_TC, 64>() || !f8_attr<moe::tc::EPI_SCALE_TC, 64>() ||
-        !f8_attr<moe::tc::EPI_SWIGLU_TC, 32>() || !f8_attr<moe::tc::EPI_SCALE_TC, 32>())
-      return MOE_ERR_CUDA;
+    if (!f8_attrs<moe::tcf8::WQ_FP8>() || !f8_attrs<moe::tcf8::WQ_MXFP4>()) return MOE_ERR_CUDA;
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
         !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
+      return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(moe::rtc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             moe::rtc::SMEM_BYTES) != cudaSuccess)
       return MOE_ERR_CUDA;
     const int rs = static_cast<int>(moe::route_smem_bytes(moe::tc::MAX_E));
     if (cudaFuncSetAttribute(moe::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -312,16 +360,16 @@ bool encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, 
   return r == CUDA_SUCCESS;
 }
 
-// FP8 code tensor map over [outer][mid][inner] codes (inner a multiple of 16),
-// box {128 codes, box_rows, 1} (full 128-byte lines), 128-byte swizzle. The
-// codes are described to the TMA unit as 32-bit words (4 codes each): the
-// bytes land exactly where a uint8 map would put them, in a quarter of the
-// elements.
+// Weight-code tensor map over [outer][mid][inner] bytes (inner a multiple of
+// 16: FP8 codes, or MXFP4 codes two per byte), box {128 bytes, box_rows, 1}
+// (full 128-byte lines), 128-byte swizzle. The bytes are described to the TMA
+// unit as 32-bit words: they land exactly where a uint8 map would put them, in
+// a quarter of the elements.
 bool encode_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
                    uint32_t box_rows) {
   cuuint64_t dims[3] = {inner / 4, mid, outer};
   cuuint64_t strides[2] = {inner, inner * mid};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::tcf8::F8Shape<128>::QK / 4), box_rows, 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::tcf8::F8Shape<128>::Q_ROW / 4), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r =
       g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box,
@@ -343,7 +391,8 @@ moe_status launched() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_
 template <typename TX>
 moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const TX* x,
                                     const float* W_r, uint8_t* ws, int32_t* counts, float* aux,
-                                    cudaStream_t st, const Timer& tm) {
+                                    cudaStream_t st, const Timer& tm,
+                                    unsigned long long wait_tmo) {
   float* logits = reinterpret_cast<float*>(ws + P.o_logits);
   int32_t* idx = reinterpret_cast<int32_t*>(ws + P.o_idx);
   float* gate = reinterpret_cast<float*>(ws + P.o_gate);
@@ -359,9 +408,33 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   TX* xp = reinterpret_cast<TX*>(ws + P.o_xp);
   const int T = static_cast<int>(P.T);
 
-  // (0) router logits, fp32 FMA
+  // (0) router logits: split-precision tensor cores (bf16 x), or fp32 FMA
   tm.at(0);
-  if (P.router_narrow) {
+  if (P.router_tc) {
+    __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + P.o_wsplit);
+    const int64_t n = static_cast<int64_t>(P.E) * P.d;
+    const int64_t blocks = (n + 255) / 256;
+    moe::rtc::split_router_weights_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096),
+                                            256, 0, st>>>(W_r, n, wsplit);
+    moe::rtc::RtcMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!encode_map(&maps.x, x, P.d, P.T, 1, moe::rtc::BM, 2) ||
+        !encode_map(&maps.w, wsplit, P.d, P.E, 3, P.router_n, 3))
+      return MOE_ERR_CUDA;
+    moe::rtc::RtcParams rp{};
+    rp.T = T;
+    rp.E = P.E;
+    rp.N = P.router_n;
+    rp.k_blocks = P.d / moe::rtc::BK / P.router_split;
+    rp.logits = logits;
+    rp.timeout_ns = wait_tmo;
+    rp.drain_timeout_ns = kDrainTimeoutNs;
+    rp.call_err = reinterpret_cast<int*>(ws + P.o_status);
+    dim3 grid((T + moe::rtc::BM - 1) / moe::rtc::BM, (P.E + P.router_n - 1) / P.router_n,
+              P.router_split);
+    moe::rtc::router_tc_kernel<<<grid, moe::rtc::NUM_THREADS, moe::rtc::SMEM_BYTES, st>>>(maps,
+                                                                                          rp);
+  } else if (P.router_narrow) {
     if (P.E <= 8) {
       dim3 grid((T + moe::NarrowShape<8>::TB - 1) / moe::NarrowShape<8>::TB, P.router_split);
       moe::router_narrow_kernel<TX, 8>
@@ -427,7 +500,8 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
       moe::scatter_kernel<uint8_t><<<qgrid, 256, 0, st>>>(
           xq, P.d, T, P.k, P.E, P.C, idx, gate, lrank, base, tile_start, slot, rowgate,
           reinterpret_cast<uint8_t*>(xp), P.rows_max, sx, reinterpret_cast<float*>(ws + P.o_xsc));
-    } else if (dims->weight_format == MOE_WEIGHTS_FP8) {  // the FP8-weight GEMMs read fp16 rows
+    } else if (dims->weight_format == MOE_WEIGHTS_FP8 || dims->weight_format == MOE_WEIGHTS_MXFP4) {
+      // the quantised-weight GEMMs read fp16 rows
       moe::scatter_kernel<TX, true><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate,
                                                           lrank, base, tile_start, slot, rowgate,
                                                           xp, P.rows_max);
@@ -467,6 +541,9 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   if (dims->weight_format != MOE_WEIGHTS_DTYPE &&
       (dims->weight_scales == nullptr || !aligned(dims->weight_scales, 4)))
     return MOE_ERR_INVALID_ARG;
+  if (dims->weight_format == MOE_WEIGHTS_MXFP4 &&
+      (dims->weight_block_scales == nullptr || !aligned(dims->weight_block_scales, 16)))
+    return MOE_ERR_INVALID_ARG;
 
   const Plan P = make_plan(dims, E, k, cf);
   if (dims->workspace == nullptr || !aligned(dims->workspace, 256) ||
@@ -491,7 +568,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   if (P.bf16) {
     using bf16 = __nv_bfloat16;
     s = launch_route_and_permute<bf16>(P, dims, static_cast<const bf16*>(x), W_r, ws, counts, aux,
-                                       st, tm);
+                                       st, tm, wait_tmo);
     if (s != MOE_OK) return s;
     const bf16* xp = reinterpret_cast<const bf16*>(ws + P.o_xp);
     bf16* h = reinterpret_cast<bf16*>(ws + P.o_h);
@@ -543,27 +620,34 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tm.at(9);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
       tm.at(10);
-      moe::tcf8::quantize_rows_fp8_kernel<bf16>
+      moe::tcf8::quantize_rows_fp8_kernel<float>
           <<<static_cast<unsigned>(P.rows_max < 8192 ? P.rows_max : 8192), 256, 0, st>>>(
-              h, P.rows_max, P.de, hq, hsc, tile_start, counts, E, P.C);
+              reinterpret_cast<const float*>(h), P.rows_max, P.de, hq, hsc, tile_start, counts, E,
+              P.C);
       launch_tc<moe::tc::EPI_SCALE_TC, true>(arows, num_sms, st, dn, td);
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
-    } else if (dims->weight_format == MOE_WEIGHTS_FP8) {
-      // FP8 expert weights: 1-CTA kernels that dequantise the weight tiles on chip
+    } else if (dims->weight_format == MOE_WEIGHTS_FP8 || dims->weight_format == MOE_WEIGHTS_MXFP4) {
+      // FP8 or MXFP4 expert weights: 1-CTA kernels that dequantise the weight
+      // tiles on chip
+      const bool mx = dims->weight_format == MOE_WEIGHTS_MXFP4;
       const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
       const float* sc = dims->weight_scales;
       const size_t gsz = static_cast<size_t>(E) * P.de;
+      const int cpb = mx ? 2 : 1;  // codes per byte
       moe::tc::TcMaps up, dn;
       memset(&up, 0, sizeof(up));
       memset(&dn, 0, sizeof(dn));
       const bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, arows, 2) &&
-                      encode_map_u8(&up.b0[0], W_g, P.d, P.de, E, moe::tc::BN / 2) &&
-                      encode_map_u8(&up.b1[0], W_u, P.d, P.de, E, moe::tc::BN / 2) &&
+                      encode_map_u8(&up.b0[0], W_g, P.d / cpb, P.de, E, moe::tc::BN / 2) &&
+                      encode_map_u8(&up.b1[0], W_u, P.d / cpb, P.de, E, moe::tc::BN / 2) &&
                       encode_map(&dn.a[0], h, P.de, P.rows_max, 1, arows, 2) &&
-                      encode_map_u8(&dn.b0[0], W_d, P.de, P.d, E, moe::tc::BN);
+                      encode_map_u8(&dn.b0[0], W_d, P.de / cpb, P.d, E, moe::tc::BN);
       if (!ok) return MOE_ERR_CUDA;
       dn.b1[0] = dn.b0[0];
+      // MXFP4 block exponents: [W_g | W_u | W_d], K / 32 bytes per weight row
+      const uint8_t* bs = dims->weight_block_scales;
+      const size_t gbs = gsz * (P.d / 32);
       moe::tcf8::F8Params fu{};
       fu.timeout_ns = wait_tmo;
       fu.drain_timeout_ns = kDrainTimeoutNs;
@@ -573,21 +657,39 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       fu.grp.scale0 = sc;
       fu.grp.scale1 = sc + gsz;
       fu.grp.scale_stride = P.de;
+      if (mx) {
+        fu.grp.bscale0 = bs;
+        fu.grp.bscale1 = bs + gbs;
+        fu.grp.bscale_stride = static_cast<int64_t>(P.de) * (P.d / 32);
+        fu.grp.kblk = P.d / 32;
+      }
       moe::tcf8::F8Params fd{};
       fd.timeout_ns = wait_tmo;
       fd.drain_timeout_ns = kDrainTimeoutNs;
       fd.call_err = call_err;
-      fd.grp.g = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN, P.de / moe::tc::BK,
-                  P.d, yrows, rowgate};
+      fd.grp.g = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN,
+                  P.de / moe::tc::BK, P.d, yrows, rowgate};
       fd.grp.scale0 = sc + 2 * gsz;
       fd.grp.scale1 = sc + 2 * gsz;
       fd.grp.scale_stride = P.d;
+      if (mx) {
+        fd.grp.bscale0 = bs + 2 * gbs;
+        fd.grp.bscale1 = bs + 2 * gbs;
+        fd.grp.bscale_stride = static_cast<int64_t>(P.d) * (P.de / 32);
+        fd.grp.kblk = P.de / 32;
+      }
       tm.at(8);
-      launch_f8<moe::tc::EPI_SWIGLU_TC>(arows, num_sms, st, up, fu);
+      if (mx)
+        launch_f8<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>(arows, num_sms, st, up, fu);
+      else
+        launch_f8<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_FP8>(arows, num_sms, st, up, fu);
       tm.at(9);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
       tm.at(10);
-      launch_f8<moe::tc::EPI_SCALE_TC>(arows, num_sms, st, dn, fd);
+      if (mx)
+        launch_f8<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_MXFP4>(arows, num_sms, st, dn, fd);
+      else
+        launch_f8<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>(arows, num_sms, st, dn, fd);
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     } else {
@@ -717,7 +819,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
 
   // fp32 layer: the same pipeline with fp32 FMA expert products
   const float* xf = static_cast<const float*>(x);
-  s = launch_route_and_permute<float>(P, dims, xf, W_r, ws, counts, aux, st, tm);
+  s = launch_route_and_permute<float>(P, dims, xf, W_r, ws, counts, aux, st, tm, wait_tmo);
   if (s != MOE_OK) return s;
   const float* xp = reinterpret_cast<const float*>(ws + P.o_xp);
   float* h = reinterpret_cast<float*>(ws + P.o_h);
@@ -901,6 +1003,41 @@ moe_status moe_dequantize_fp8(const uint8_t* codes, const float* scales, int64_t
   moe::tcf8::dequantize_rows_fp8_kernel<<<static_cast<unsigned>(blocks < 16384 ? blocks : 16384),
                                           256, 0, static_cast<cudaStream_t>(stream)>>>(
       codes, scales, rows, cols, out);
+  return launched();
+}
+
+moe_status moe_quantize_mxfp4(const void* w, int32_t dtype, int64_t rows, int32_t cols,
+                              uint8_t* codes, uint8_t* block_scales, float* row_factors,
+                              void* stream) {
+  if (w == nullptr || codes == nullptr || block_scales == nullptr || row_factors == nullptr ||
+      rows < 0 || cols < 1 || cols % 32 != 0 || (dtype != MOE_BF16 && dtype != MOE_F32) ||
+      !aligned(w, 16) || !aligned(codes, 16) || !aligned(row_factors, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(rows < 8192 ? rows : 8192);
+  if (dtype == MOE_BF16)
+    moe::tcf8::quantize_rows_mxfp4_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), rows, cols, codes, block_scales, row_factors);
+  else
+    moe::tcf8::quantize_rows_mxfp4_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float*>(w), rows, cols, codes, block_scales, row_factors);
+  return launched();
+}
+
+moe_status moe_dequantize_mxfp4(const uint8_t* codes, const uint8_t* block_scales,
+                                const float* row_factors, int64_t rows, int32_t cols, float* out,
+                                void* stream) {
+  if (codes == nullptr || block_scales == nullptr || row_factors == nullptr || out == nullptr ||
+      rows < 0 || cols < 1 || cols % 32 != 0 || !aligned(codes, 16) || !aligned(out, 16) ||
+      !aligned(row_factors, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  const int64_t n = rows * (cols / 16);
+  const int64_t blocks = (n + 255) / 256;
+  moe::tcf8::dequantize_rows_mxfp4_kernel<<<static_cast<unsigned>(blocks < 16384 ? blocks : 16384),
+                                            256, 0, static_cast<cudaStream_t>(stream)>>>(
+      codes, block_scales, row_factors, rows, cols, out);
   return launched();
 }
 

@@ -66,13 +66,15 @@ constexpr int CONV_WARP0 = 6;
 enum { WQ_FP8 = 0, WQ_MXFP4 = 1 };
 
 // Ring shape for an activation box of AR rows and weight format WQ. For small
-// boxes (weight-streaming shapes) a stage is one 64-deep chunk and the code
-// ring is four deep, so up to 128 KB of codes per SM are in flight while the
-// decoded tiles turn over; for 128-row boxes the decoded ring is deeper.
+// boxes (weight-streaming shapes) a stage is two 64-deep chunks: each stage
+// hand-off between converters and the MMA thread costs a roughly fixed
+// latency, so fewer, larger stages stream faster (measured: one chunk per stage
+// with a four-deep code ring took about 2000 cycles per chunk, two chunks per
+// stage about 1400). For 128-row boxes a stage is one chunk.
 template <int AR, int WQ = WQ_FP8>
 struct F8Shape {
   static_assert(AR == 128 || AR == 64 || AR == 32, "activation box rows");
-  static constexpr int CH = 1;                       // 64-deep K chunks per stage
+  static constexpr int CH = AR == 128 ? 1 : 2;       // 64-deep K chunks per stage
   static constexpr int A_SUB = AR * BK * 2;          // fp16 activation box of one chunk
   static constexpr int B_SUB = BN * BK * 2;          // decoded fp16 weights of one chunk
   static constexpr int A_BYTES = CH * A_SUB;         // a stage of ring A
@@ -82,8 +84,8 @@ struct F8Shape {
   static constexpr int QCH = QK / BK;                // 64-deep chunks per Q stage
   static constexpr int Q_BYTES = BN * Q_ROW;         // 256 rows x 128 B
   static constexpr int NS = AR == 128 ? 3 : 2;
-  static constexpr int NA = 4;                       // activations run ahead of the weights
-  static constexpr int NQ = AR == 128 ? 2 : 4;
+  static constexpr int NA = AR == 64 ? 2 : 4;        // activations run ahead of the weights
+  static constexpr int NQ = 2;
   static constexpr int RING_BYTES = NS * S_BYTES + NA * A_BYTES + NQ * Q_BYTES;
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");

@@ -8,7 +8,8 @@
 // Two epilogues:
 //   SwiGLU (gate/up projection): each 256-column accumulator tile holds 128
 //     gate columns (x W_g) followed by the matching 128 up columns (x W_u);
-//     the epilogue writes H = SiLU(gate) * up as bf16.
+//     the epilogue writes H = SiLU(gate) * up as bf16 (fp32 with E4M3
+//     operands, for the per-row quantiser of H that follows).
 //   Scale (down projection): Yrows = g_row * (H W_d) as bf16, g_row the gate
 //     of the assignment that owns the row (1 for the shared expert).
 // Sources: Zero to Frontier 13.1 "Why MoE", "The MoE layer" (SwiGLU experts,
@@ -545,7 +546,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 h[i] = silu_f32(a) * b;
               }
-              st_v4(out + col0 + q * 8, Vec16<__nv_bfloat16>::pack(h));
+              if (Q8) {
+                // E4M3 operands: H stays fp32, so that the per-row quantiser that
+                // follows decides its codes from H itself, not from a bf16 copy
+                float* o32 = reinterpret_cast<float*>(g.out) + (size_t)row * g.N + col0 + q * 8;
+                st_v4(o32, Vec16<float>::pack(h));
+                st_v4(o32 + 4, Vec16<float>::pack(h + 4));
+              } else {
+                st_v4(out + col0 + q * 8, Vec16<__nv_bfloat16>::pack(h));
+              }
             }
           }
         }

@@ -83,6 +83,10 @@ DECODE_PROFILE = Workload("decode-shape-profile T=32 d=4096 E=2 d_e=14336 k=2",
 # experts, so the whole case holds about 0.2 GB, for hardware-counter captures.
 ROUTING_PROFILE = Workload("routing-kernels-profile T=4096 d=4096 E=8 d_e=256 k=2",
                            4096, 4096, 8, 256, 2, seed=1)
+# The DeepSeek-V3-shaped router (T, d, E and k of that layer) with narrow
+# experts, about 1 GB on the device.
+DSV3_ROUTING_PROFILE = Workload("dsv3-routing-profile T=8192 d=7168 E=256 d_e=64 k=8",
+                                8192, 7168, 256, 64, 8, seed=2)
 
 
 def zipf_router_bias(E: int) -> torch.Tensor:

@@ -32,13 +32,15 @@ class Workspace:
 
 def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, stream, events,
               wait_timeout_ns: int = 0, routing: Optional[dict] = None, weight_scales=None,
-              act_fp8: bool = False):
+              act_fp8: bool = False, weight_block_scales=None):
     T, d = x.shape
     d_e = W_g.shape[1]
     routing = routing or {}
     fmt = _lib.MOE_WEIGHTS_DTYPE
     if W_g.dtype == torch.uint8:
         fmt = _lib.MOE_WEIGHTS_FP8_W8A8 if act_fp8 else _lib.MOE_WEIGHTS_FP8
+        if weight_block_scales is not None:
+            fmt = _lib.MOE_WEIGHTS_MXFP4
     return _lib.make_dims(T, d, d_e, d_s, dtype_code(x.dtype), router_bias, ws,
                           ws.numel() if ws is not None else 0, stream, events,
                           wait_timeout_ns=wait_timeout_ns,
@@ -46,7 +48,8 @@ def _dims_for(x: torch.Tensor, W_g: torch.Tensor, d_s: int, router_bias, ws, str
                           selection_bias=routing.get("selection_bias"),
                           n_group=routing.get("n_group", 0),
                           topk_group=routing.get("topk_group", 0),
-                          weight_format=fmt, weight_scales=weight_scales)
+                          weight_format=fmt, weight_scales=weight_scales,
+                          weight_block_scales=weight_block_scales)
 
 
 def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Tensor,
@@ -57,7 +60,7 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
             counts: Optional[torch.Tensor] = None, wait_timeout_ns: int = 0,
             gate_mode: int = 0, selection_bias: Optional[torch.Tensor] = None,
             n_group: int = 0, topk_group: int = 0, weight_scales: Optional[torch.Tensor] = None,
-            act_fp8: bool = False):
+            act_fp8: bool = False, weight_block_scales: Optional[torch.Tensor] = None):
     """Run the routed MoE FFN layer; returns (y, aux[1] fp32, counts[E] int32) on x's device.
 
     Shapes: x [T, d]; W_r [E, d] fp32; W_g, W_u [E, d_e, d]; W_d [E, d, d_e];
@@ -66,6 +69,9 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
     weight_scales = their per-row scales concatenated [W_g | W_u | W_d] (bf16 x).
     act_fp8 (with FP8 weights): E4M3 activations inside the experts as well
     (MOE_WEIGHTS_FP8_W8A8 in include/moe.h).
+    MXFP4 expert weights: W_g, W_u, W_d as packed uint8 E2M1 codes [.., K / 2]
+    (quantize_mxfp4), weight_block_scales = their E8M0 block scales and
+    weight_scales = their row factors, each concatenated [W_g | W_u | W_d].
     wait_timeout_ns: limit of the GEMM kernels' device-side waits (0 = library default).
     gate_mode / selection_bias / n_group / topk_group: routing variants (include/moe.h).
     """
@@ -88,14 +94,17 @@ def forward(x: torch.Tensor, W_r: torch.Tensor, W_g: torch.Tensor, W_u: torch.Te
             raise RuntimeError("FP8 weights need weight_scales: a CUDA fp32 tensor")
     elif act_fp8:
         raise RuntimeError("act_fp8 needs FP8 (uint8) weights")
+    if weight_block_scales is not None and (act_fp8 or W_g.dtype != torch.uint8):
+        raise RuntimeError("weight_block_scales go with MXFP4 (uint8) weights, without act_fp8")
     probe = _dims_for(x, W_g, d_s, router_bias, None, stream, events, routing=routing,
-                      weight_scales=weight_scales, act_fp8=act_fp8)
+                      weight_scales=weight_scales, act_fp8=act_fp8,
+                      weight_block_scales=weight_block_scales)
     nbytes = _lib.moe_workspace_size(probe, E, k, capacity_factor)
     if nbytes == 0:
         raise _lib.MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
     ws = workspace.get(nbytes, dev)
     dims = _dims_for(x, W_g, d_s, router_bias, ws, stream, events, wait_timeout_ns, routing,
-                     weight_scales, act_fp8)
+                     weight_scales, act_fp8, weight_block_scales)
     y = torch.empty_like(x) if y is None else y
     aux = torch.empty(1, dtype=torch.float32, device=dev) if aux is None else aux
     counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
@@ -128,6 +137,38 @@ def dequantize_fp8(codes: torch.Tensor, scales: torch.Tensor, stream=None) -> to
     rc = _lib.moe_dequantize_fp8(codes, scales, rows, cols, out, st)
     if rc != _lib.MOE_OK:
         raise _lib.MoeError(rc, "moe_dequantize_fp8")
+    return out
+
+
+def quantize_mxfp4(w: torch.Tensor, stream=None):
+    """MXFP4 codes (uint8, w's shape with the last dimension halved), E8M0 block
+    scales (uint8, last dimension / 32) and fp32 row factors (w's shape without
+    the last dimension) of a CUDA weight tensor whose last dimension is the row
+    (include/moe.h, moe_quantize_mxfp4)."""
+    if not w.is_cuda or not w.is_contiguous():
+        raise RuntimeError("w must be a contiguous CUDA tensor")
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    codes = torch.empty(*w.shape[:-1], cols // 2, dtype=torch.uint8, device=w.device)
+    bscales = torch.empty(*w.shape[:-1], cols // 32, dtype=torch.uint8, device=w.device)
+    factors = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    st = torch.cuda.current_stream(w.device).cuda_stream if stream is None else stream
+    rc = _lib.moe_quantize_mxfp4(w, dtype_code(w.dtype), rows, cols, codes, bscales, factors, st)
+    if rc != _lib.MOE_OK:
+        raise _lib.MoeError(rc, "moe_quantize_mxfp4")
+    return codes, bscales, factors
+
+
+def dequantize_mxfp4(codes: torch.Tensor, bscales: torch.Tensor, factors: torch.Tensor,
+                     stream=None) -> torch.Tensor:
+    """fp32 weights code * 2^X, as the MXFP4 layer computes with them (moe_dequantize_mxfp4)."""
+    cols = codes.shape[-1] * 2
+    rows = codes.numel() * 2 // cols
+    out = torch.empty(*codes.shape[:-1], cols, dtype=torch.float32, device=codes.device)
+    st = torch.cuda.current_stream(codes.device).cuda_stream if stream is None else stream
+    rc = _lib.moe_dequantize_mxfp4(codes, bscales, factors, rows, cols, out, st)
+    if rc != _lib.MOE_OK:
+        raise _lib.MoeError(rc, "moe_dequantize_mxfp4")
     return out
 
 

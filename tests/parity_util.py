@@ -27,7 +27,8 @@ def run_gpu(w: Workload, inp: dict, ws: Workspace | None = None, fp8: dict | Non
                              gate_mode=w.gate_mode, selection_bias=inp.get("selection_bias"),
                              n_group=w.n_group, topk_group=w.topk_group,
                              weight_scales=fp8["weight_scales"] if fp8 is not None else None,
-                             act_fp8=act_fp8)
+                             act_fp8=act_fp8,
+                             weight_block_scales=fp8.get("block_scales") if fp8 else None)
     torch.cuda.synchronize()
     assert moe_get_device_status() == 0, "a device-side wait timed out"
     views = routing_views(ws.buf, inp["x"], src["W_g"], w.E, w.k, w.capacity_factor, w.d_s,
@@ -45,6 +46,8 @@ def run_oracle(w: Workload, inp: dict, rows=None, fp8: dict | None = None,
     def expert(e):
         if fp8 is None:
             return inp["W_g"][e].cpu(), inp["W_u"][e].cpu(), inp["W_d"][e].cpu()
+        if "oracle_mx" in fp8:  # MXFP4: the oracle's own codes and block exponents
+            return tuple(O.dequantize_rows_mxfp4(c[e], x[e]) for c, x in fp8["oracle_mx"])
         E, de, d = w.E, w.d_e, w.d
         sc = fp8["weight_scales"]
         parts = ((fp8["W_g"][e], sc[e * de:(e + 1) * de]),
@@ -222,3 +225,36 @@ def oracle_quantized_weights(inp: dict, device="cuda") -> dict:
         scales.append(torch.from_numpy(sc))
     out["weight_scales"] = torch.cat(scales).to(device)
     return out
+
+
+def pack_e2m1(codes: np.ndarray) -> np.ndarray:
+    """One 4-bit code per element -> two per byte, the even element in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def oracle_mxfp4_weights(inp: dict, device="cuda") -> dict:
+    """MXFP4 codes, block scales and row factors of the drawn dtype weights,
+    quantised by the oracle on the CPU, in the layer's input layout; also the
+    oracle's own (codes, exponents) per stack for its reference."""
+    out, bsc, rfs, mx = {}, [], [], []
+    for name in ("W_g", "W_u", "W_d"):
+        wt = inp[name].float().cpu().numpy()
+        n, r, c = wt.shape
+        codes, exps = O.quantize_rows_mxfp4(wt.reshape(-1, c))
+        out[name] = torch.from_numpy(pack_e2m1(codes).reshape(n, r, c // 2)).to(device)
+        bsc.append(torch.from_numpy((exps + 127).astype(np.uint8).reshape(-1)))
+        rfs.append(torch.from_numpy(row_factors_of(codes, exps)))
+        mx.append((codes.reshape(n, r, c), exps.reshape(n, r, c // 32)))
+    out["block_scales"] = torch.cat(bsc).to(device)
+    out["weight_scales"] = torch.cat(rfs).to(device)
+    out["oracle_mx"] = mx
+    return out
+
+
+def row_factors_of(codes: np.ndarray, exps: np.ndarray) -> np.ndarray:
+    """2^(largest exponent among each row's blocks that hold a non-zero code), 1 if none."""
+    rows, K = codes.shape
+    nz = (codes.reshape(rows, K // 32, 32) & 0x7).any(axis=2)
+    big = np.where(nz, exps, np.iinfo(np.int64).min).max(axis=1)
+    return np.where(nz.any(axis=1), np.ldexp(1.0, np.maximum(big, -200)), 1.0).astype(np.float32)

@@ -118,7 +118,10 @@ def test_workspace_size_and_layout(lib):
     (8, 2, dict(weight_format=1, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),  # FP8: bf16 x
     (8, 2, dict(weight_format=1, d_s=128), _lib.MOE_ERR_UNSUPPORTED),  # FP8: no shared expert
     (8, 2, dict(weight_format=2, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),  # W8A8: bf16 x
-    (8, 2, dict(weight_format=3), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(weight_format=4), _lib.MOE_ERR_INVALID_ARG),
+    (8, 2, dict(weight_format=3, d=320), _lib.MOE_ERR_UNSUPPORTED),    # MXFP4: d % 256
+    (8, 2, dict(weight_format=3, d_e=192), _lib.MOE_ERR_UNSUPPORTED),  # MXFP4: d_e % 256
+    (8, 2, dict(weight_format=3, d_s=256), _lib.MOE_ERR_UNSUPPORTED),  # MXFP4: no shared
 ])
 def test_forward_rejects_bad_shapes_on_host(lib, E, k, kw, want):
     d = _dims(**kw)
@@ -194,6 +197,30 @@ def test_fp8_weights_validated_on_host(lib):
                  (g + 8, g, 4, 64, g), (g, g, 4, 64, g + 4), (g, g, -2, 64, g)]:
         assert _lib.moe_dequantize_fp8(*args) == _lib.MOE_ERR_INVALID_ARG, args
     assert _lib.moe_dequantize_fp8(g, g, 0, 64, g) == _lib.MOE_OK
+
+
+def test_mxfp4_weights_validated_on_host(lib):
+    g = 1 << 20
+    fwd = lambda d: _lib.moe_forward(d, g, g, g, g, g, None, 8, 2, 0.0, g, g, g, check=False)
+    mx = dict(weight_format=3, weight_scales=g, weight_block_scales=g)
+    assert fwd(_dims(**mx)) == _lib.MOE_ERR_WORKSPACE                     # valid
+    assert fwd(_dims(**dict(mx, weight_block_scales=None))) == _lib.MOE_ERR_INVALID_ARG
+    assert fwd(_dims(**dict(mx, weight_block_scales=g + 8))) == _lib.MOE_ERR_INVALID_ARG
+    assert fwd(_dims(**dict(mx, weight_scales=None))) == _lib.MOE_ERR_INVALID_ARG
+    assert fwd(_dims(**dict(mx, dtype=_lib.MOE_F32))) == _lib.MOE_ERR_UNSUPPORTED
+    # the same workspace as FP8 weight-only (no activation codes)
+    assert _lib.moe_workspace_size(_dims(**mx), 8, 2, 0.0) == \
+        _lib.moe_workspace_size(_dims(weight_format=1), 8, 2, 0.0)
+    for args in [(0, 1, 4, 64, g, g, g), (g, 1, 4, 64, 0, g, g), (g, 1, 4, 64, g, 0, g),
+                 (g, 1, 4, 64, g, g, 0), (g, 1, 4, 48, g, g, g), (g, 1, -1, 64, g, g, g),
+                 (g, 9, 4, 64, g, g, g), (g + 8, 1, 4, 64, g, g, g), (g, 1, 4, 64, g + 8, g, g)]:
+        assert _lib.moe_quantize_mxfp4(*args) == _lib.MOE_ERR_INVALID_ARG, args
+    assert _lib.moe_quantize_mxfp4(g, 1, 0, 64, g, g, g) == _lib.MOE_OK
+    for args in [(0, g, g, 4, 64, g), (g, 0, g, 4, 64, g), (g, g, 0, 4, 64, g),
+                 (g, g, g, 4, 64, 0), (g, g, g, 4, 40, g), (g + 8, g, g, 4, 64, g),
+                 (g, g, g, 4, 64, g + 4), (g, g, g, -1, 64, g)]:
+        assert _lib.moe_dequantize_mxfp4(*args) == _lib.MOE_ERR_INVALID_ARG, args
+    assert _lib.moe_dequantize_mxfp4(g, g, g, 0, 64, g) == _lib.MOE_OK
 
 
 def test_binding_refuses_cpu_tensors():

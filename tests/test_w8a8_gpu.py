@@ -3,9 +3,9 @@
 * The E4M3 activation rows the layer builds: the codes and scales of every
   kept x row bit-exact against the oracle's per-row quantiser (both decide in
   fp32 from the same bf16 values).
-* The hidden rows' codes: the layer decides them from its own fp32 H rounded
-  to bf16, the oracle from its fp64 H rounded the same way, so a code may flip
-  where H sits on a rounding boundary; almost all must agree.
+* The hidden rows' codes: the layer decides them from its own fp32 H, the
+  oracle from its fp64 H, so a code may flip where H sits within fp32
+  accumulation error of a rounding boundary; almost all must agree.
 * y against the oracle's W8A8 expert within the bf16 tolerance, routing exact,
   over the three activation-box sizes, N and K tails, many experts, capacity,
   random codes, and the full-size decode and (sampled) Mixtral shapes.
@@ -82,12 +82,12 @@ def test_w8a8_hidden_codes_mostly_agree():
         Wg = O.dequantize_rows_fp8(fp8["W_g"][e].cpu().numpy(), sc[e * de:(e + 1) * de])
         Wu = O.dequantize_rows_fp8(fp8["W_u"][e].cpu().numpy(), sc[E * de + e * de:E * de + (e + 1) * de])
         xq = O.fake_quant_rows_fp8(x[toks])
-        h = O.round_bf16(O.silu(xq @ Wg.T) * (xq @ Wu.T))
+        h = O.silu(xq @ Wg.T) * (xq @ Wu.T)
         codes, _ = O.quantize_rows_fp8(h)
         got = hq[slot[toks, 0]]
         agree += int((got == codes).sum())
         total += codes.size
-    assert total > 0 and agree / total > 0.995, agree / total
+    assert total > 0 and agree / total > 0.999, agree / total
 
 
 def test_w8a8_random_codes():
