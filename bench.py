@@ -356,10 +356,16 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device-side wait timed out during warm-up")
 
     barrier()
-    ms, clk = time_calls(lambda i, ev: call_on(xs, y, i, ev), args.steps, stream, kev, local_rank)
+    ms, clk = time_calls(lambda i, ev: call_on(xs, y, i, None), args.steps, stream, None,
+                         local_rank)
     barrier()
     if moe_get_device_status() != 0:
         raise RuntimeError("device-side wait timed out in the timed region")
+    # per-kernel breakdown: the same steps again, with the library's events around
+    # each kernel (events between kernels stop them overlapping their launches,
+    # so these steps are not part of the value's timing)
+    time_calls(lambda i, ev: call_on(xs, y, i, ev), args.steps, stream, kev, local_rank)
+    barrier()
     per_kernel = [statistics.mean(kev[i].elapsed_ms(j) for i in range(args.steps))
                   for j in range(MOE_NUM_KERNELS)]
     for kv in kev:
@@ -519,10 +525,12 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         dkev = [KernelEvents(MOE_NUM_KERNELS) for _ in range(n)]
         barrier()
-        dms, dclk = time_calls(dcall, n, stream, dkev, local_rank)
+        dms, dclk = time_calls(lambda i, ev: dcall(i, None), n, stream, None, local_rank)
         barrier()
         if moe_get_device_status() != 0:
             raise RuntimeError("device-side wait timed out in the decode leg")
+        time_calls(dcall, n, stream, dkev, local_rank)  # per-kernel breakdown, as above
+        barrier()
         dk = [statistics.mean(dkev[i].elapsed_ms(j) for i in range(n))
               for j in range(MOE_NUM_KERNELS)]
         for kv in dkev:

@@ -22,6 +22,19 @@ constexpr int DEVERR_BOUNDS = 2;
 // kernel between a separate read and clear cannot be lost.
 __global__ void take_device_error_kernel() { g_dev_error_taken = atomicExch(&g_dev_error, 0); }
 
+// Programmatic dependent launch: the kernels of a forward pass are launched
+// while the previous kernel in the stream is still finishing, so that launch
+// latency and set-up (barriers, TMEM, tensor-map prefetch) overlap its tail.
+// pdl_wait() blocks until the previous kernel has completed and its memory is
+// visible; every kernel calls it in all threads before its first global
+// memory access that another kernel (of this pass, the previous pass, or the
+// caller's work before it) may make. pdl_launch_dependents() then lets the
+// next kernel start launching. Both are no-ops for a plain launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Record a failed bounds check (MOE_DEBUG builds).
 __device__ __forceinline__ void flag_bounds() { atomicOr(&g_dev_error, DEVERR_BOUNDS); }
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <mutex>
+#include <utility>
 #include <string.h>
 
 #include "moe.h"
@@ -193,6 +194,26 @@ bool tc_attr() {
                               moe::tc::TcShape<AR>::SMEM_BYTES) == cudaSuccess;
 }
 
+// Launch a kernel of the forward pass with programmatic dependent launch: it
+// may start launching while the previous kernel in the stream finishes, and
+// waits in the kernel (pdl_wait) before touching memory that kernel may use.
+// A failure is left for launched() to report.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int EPI, int AR, int WQ>
 bool f8_attr() {
   return cudaFuncSetAttribute(moe::tcf8::tc_f8_grouped_gemm_kernel<EPI, AR, WQ>,
@@ -216,14 +237,11 @@ void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
                const moe::tcf8::F8Params& fp) {
   using namespace moe::tcf8;
   if (ar == 32)
-    tc_f8_grouped_gemm_kernel<EPI, 32, WQ>
-        <<<grid, NUM_THREADS, F8Shape<32, WQ>::SMEM_BYTES, st>>>(maps, fp);
+    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 32, WQ>, grid, NUM_THREADS, F8Shape<32, WQ>::SMEM_BYTES, st, maps, fp);
   else if (ar == 64)
-    tc_f8_grouped_gemm_kernel<EPI, 64, WQ>
-        <<<grid, NUM_THREADS, F8Shape<64, WQ>::SMEM_BYTES, st>>>(maps, fp);
+    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 64, WQ>, grid, NUM_THREADS, F8Shape<64, WQ>::SMEM_BYTES, st, maps, fp);
   else
-    tc_f8_grouped_gemm_kernel<EPI, 128, WQ>
-        <<<grid, NUM_THREADS, F8Shape<128, WQ>::SMEM_BYTES, st>>>(maps, fp);
+    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 128, WQ>, grid, NUM_THREADS, F8Shape<128, WQ>::SMEM_BYTES, st, maps, fp);
 }
 
 // 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32);
@@ -233,18 +251,18 @@ void launch_tc(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
                const moe::tc::TcParams& tp) {
   using namespace moe::tc;
   if (ar == 32)
-    tc_grouped_gemm_kernel<EPI, 32, Q8>
-        <<<grid, NUM_THREADS, TcShape<32>::SMEM_BYTES, st>>>(maps, tp);
+    launch_pdl(tc_grouped_gemm_kernel<EPI, 32, Q8>, grid, NUM_THREADS, TcShape<32>::SMEM_BYTES, st, maps, tp);
   else if (ar == 64)
-    tc_grouped_gemm_kernel<EPI, 64, Q8>
-        <<<grid, NUM_THREADS, TcShape<64>::SMEM_BYTES, st>>>(maps, tp);
+    launch_pdl(tc_grouped_gemm_kernel<EPI, 64, Q8>, grid, NUM_THREADS, TcShape<64>::SMEM_BYTES, st, maps, tp);
   else
-    tc_grouped_gemm_kernel<EPI, 128, Q8>
-        <<<grid, NUM_THREADS, TcShape<128>::SMEM_BYTES, st>>>(maps, tp);
+    launch_pdl(tc_grouped_gemm_kernel<EPI, 128, Q8>, grid, NUM_THREADS, TcShape<128>::SMEM_BYTES, st, maps, tp);
 }
 
+// Launch configuration of the CTA-pair kernels: clusters of two; with `pdl`,
+// also programmatic dependent launch (see launch_pdl). attr holds 2 entries.
 template <int EPI>
-cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr,
+                               bool pdl = false) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(moe::tc2::NUM_THREADS, 1, 1);
@@ -254,8 +272,10 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cfg;
 }
 
@@ -265,7 +285,7 @@ bool pair_setup(int num_sms, int* clusters) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            moe::tc2::SMEM_BYTES) != cudaSuccess)
     return false;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config<EPI>(num_sms / 2, nullptr, attr);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return false;
@@ -388,6 +408,8 @@ struct Timer {
 
 moe_status launched() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+
+
 template <typename TX>
 moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const TX* x,
                                     const float* W_r, uint8_t* ws, int32_t* counts, float* aux,
@@ -414,8 +436,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + P.o_wsplit);
     const int64_t n = static_cast<int64_t>(P.E) * P.d;
     const int64_t blocks = (n + 255) / 256;
-    moe::rtc::split_router_weights_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096),
-                                            256, 0, st>>>(W_r, n, wsplit);
+    launch_pdl(moe::rtc::split_router_weights_kernel, static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, st, W_r, n, wsplit);
     moe::rtc::RtcMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (!encode_map(&maps.x, x, P.d, P.T, 1, moe::rtc::BM, 2) ||
@@ -432,37 +453,47 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
     rp.call_err = reinterpret_cast<int*>(ws + P.o_status);
     dim3 grid((T + moe::rtc::BM - 1) / moe::rtc::BM, (P.E + P.router_n - 1) / P.router_n,
               P.router_split);
-    moe::rtc::router_tc_kernel<<<grid, moe::rtc::NUM_THREADS, moe::rtc::SMEM_BYTES, st>>>(maps,
+    launch_pdl(moe::rtc::router_tc_kernel, grid, moe::rtc::NUM_THREADS, moe::rtc::SMEM_BYTES, st, maps,
                                                                                           rp);
   } else if (P.router_narrow) {
     if (P.E <= 8) {
       dim3 grid((T + moe::NarrowShape<8>::TB - 1) / moe::NarrowShape<8>::TB, P.router_split);
-      moe::router_narrow_kernel<TX, 8>
-          <<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split, logits);
+      launch_pdl(moe::router_narrow_kernel<TX, 8>, grid, 256, 0, st, x, W_r, T, P.d, P.E, P.router_split, logits);
     } else {
       dim3 grid((T + moe::NarrowShape<16>::TB - 1) / moe::NarrowShape<16>::TB, P.router_split);
-      moe::router_narrow_kernel<TX, 16>
-          <<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split, logits);
+      launch_pdl(moe::router_narrow_kernel<TX, 16>, grid, 256, 0, st, x, W_r, T, P.d, P.E, P.router_split, logits);
     }
   } else {
     dim3 grid((P.E + moe::RW_BN - 1) / moe::RW_BN, (T + moe::RW_BM - 1) / moe::RW_BM,
               P.router_split);
-    moe::router_wide_kernel<TX><<<grid, 256, 0, st>>>(x, W_r, T, P.d, P.E, P.router_split,
+    launch_pdl(moe::router_wide_kernel<TX>, grid, 256, 0, st, x, W_r, T, P.d, P.E, P.router_split,
                                                        logits);
   }
   tm.at(1);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
 
-  // (1) routing
+  // (1) routing; a batch of one 64-token chunk with at most 256 experts also
+  // runs the scan (step 2) in the same kernel
+  const bool fused_scan = P.nblk == 1 && P.E <= 256;
+  moe::ScanArgs sa{};
+  sa.fused = fused_scan;
+  sa.C = P.C;
+  sa.rows_max = P.rows_max;
+  sa.counts = counts;
+  sa.base = base;
+  sa.tile_start = tile_start;
+  sa.pair_start = pair_start;
+  sa.probsum = probsum;
+  sa.aux = aux;
+  sa.call_err = reinterpret_cast<int*>(ws + P.o_status);
   tm.at(2);
   {
     const size_t smem = moe::route_smem_bytes(P.E);
     const int nv = (P.E + 31) / 32;
-#define MOE_ROUTE(NV)                                                                           \
-  moe::route_kernel<NV><<<P.nblk, 256, smem, st>>>(                                         \
-      logits, P.router_split, dims->router_bias, dims->selection_bias, dims->gate_mode,         \
-      dims->n_group, dims->topk_group, T, P.E, P.k, idx, \
-                                                   gate, lrank, hist, psum_part)
+#define MOE_ROUTE(NV)                                                                         \
+  launch_pdl(moe::route_kernel<NV>, P.nblk, 256, smem, st, \
+      logits, P.router_split, dims->router_bias, dims->selection_bias, dims->gate_mode,       \
+      dims->n_group, dims->topk_group, T, P.E, P.k, idx, gate, lrank, hist, psum_part, sa)
     if (nv <= 1) MOE_ROUTE(1);
     else if (nv <= 2) MOE_ROUTE(2);
     else if (nv <= 4) MOE_ROUTE(4);
@@ -476,10 +507,9 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
 
   // (2) scan: counts, capacity, segment offsets, aux
   tm.at(4);
-  moe::scan_kernel<<<1, 1024, 0, st>>>(hist, P.nblk, psum_part, P.nblk, P.E,
-                                       P.T, P.k, P.C, counts, base, tile_start, pair_start,
-                                       probsum, aux, reinterpret_cast<int*>(ws + P.o_status),
-                                       P.rows_max);
+  if (!fused_scan)
+    launch_pdl(moe::scan_kernel, 1, moe::scan_threads(P.E), 0, st, hist, P.nblk, psum_part, P.nblk, P.E, P.T, P.k, P.C, counts, base, tile_start, pair_start,
+        probsum, aux, sa.call_err, P.rows_max);
   tm.at(5);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;
 
@@ -493,22 +523,21 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
       // scatter the code rows and carry each row's scale to its slots
       uint8_t* xq = ws + P.o_xq;
       float* sx = reinterpret_cast<float*>(ws + P.o_sx);
-      moe::tcf8::quantize_rows_fp8_kernel<TX><<<static_cast<unsigned>(T < 8192 ? T : 8192), 256,
-                                                 0, st>>>(x, T, P.d, xq, sx);
+      launch_pdl(moe::tcf8::quantize_rows_fp8_kernel<TX>, static_cast<unsigned>(T < 8192 ? T : 8192),
+                 256, 0, st, x, T, P.d, xq, sx, nullptr, nullptr, 0, int64_t(-1));
       const int qvec = P.d / 16;
       dim3 qgrid((T + 7) / 8, (qvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
-      moe::scatter_kernel<uint8_t><<<qgrid, 256, 0, st>>>(
-          xq, P.d, T, P.k, P.E, P.C, idx, gate, lrank, base, tile_start, slot, rowgate,
+      launch_pdl(moe::scatter_kernel<uint8_t>, qgrid, 256, 0, st, xq, P.d, T, P.k, P.E, P.C, idx, gate, lrank, base, tile_start, slot, rowgate,
           reinterpret_cast<uint8_t*>(xp), P.rows_max, sx, reinterpret_cast<float*>(ws + P.o_xsc));
     } else if (dims->weight_format == MOE_WEIGHTS_FP8 || dims->weight_format == MOE_WEIGHTS_MXFP4) {
       // the quantised-weight GEMMs read fp16 rows
-      moe::scatter_kernel<TX, true><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate,
+      launch_pdl(moe::scatter_kernel<TX, true>, grid, 256, 0, st, x, P.d, T, P.k, P.E, P.C, idx, gate,
                                                           lrank, base, tile_start, slot, rowgate,
-                                                          xp, P.rows_max);
+                                                          xp, P.rows_max, nullptr, nullptr);
     } else
-      moe::scatter_kernel<TX><<<grid, 256, 0, st>>>(x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
+      launch_pdl(moe::scatter_kernel<TX>, grid, 256, 0, st, x, P.d, T, P.k, P.E, P.C, idx, gate, lrank,
                                                     base, tile_start, slot, rowgate, xp,
-                                                    P.rows_max);
+                                                    P.rows_max, nullptr, nullptr);
   }
   tm.at(7);
   return launched();
@@ -620,9 +649,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tm.at(9);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
       tm.at(10);
-      moe::tcf8::quantize_rows_fp8_kernel<float>
-          <<<static_cast<unsigned>(P.rows_max < 8192 ? P.rows_max : 8192), 256, 0, st>>>(
-              reinterpret_cast<const float*>(h), P.rows_max, P.de, hq, hsc, tile_start, counts, E,
+      launch_pdl(moe::tcf8::quantize_rows_fp8_kernel<float>, static_cast<unsigned>(P.rows_max < 8192 ? P.rows_max : 8192), 256, 0, st, reinterpret_cast<const float*>(h), P.rows_max, P.de, hq, hsc, tile_start, counts, E,
               P.C);
       launch_tc<moe::tc::EPI_SCALE_TC, true>(arows, num_sms, st, dn, td);
       tm.at(11);
@@ -713,7 +740,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     int32_t* pair_start = reinterpret_cast<int32_t*>(ws + P.o_pair_start);
     constexpr int HB = 128;  // rows of B each CTA of a pair loads
     constexpr int BNp = moe::tc2::BN;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     {
       const int brows = pair_up ? HB : moe::tc::BN / 2;
       const int abox = pair_up ? moe::tc::BM : arows;
@@ -739,7 +766,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         if (P.ds)
           tu.g[1] = {nullptr, nullptr, 1, T, (P.ds + BNp / 2 - 1) / (BNp / 2), P.d / moe::tc::BK,
                      P.ds, hs, nullptr};
-        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SWIGLU_TC>(pair_clusters[0], st, attr);
+        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SWIGLU_TC>(pair_clusters[0], st, attr, true);
         if (cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SWIGLU_TC>,
                                up, tu) != cudaSuccess)
           return MOE_ERR_CUDA;
@@ -784,7 +811,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         if (P.ds)
           td.g[1] = {nullptr, nullptr, 1, T, (P.d + BNp - 1) / BNp, P.ds / moe::tc::BK, P.d, ys,
                      nullptr};
-        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SCALE_TC>(pair_clusters[1], st, attr);
+        cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SCALE_TC>(pair_clusters[1], st, attr, true);
         if (cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
                                dn, td) != cudaSuccess)
           return MOE_ERR_CUDA;
@@ -810,7 +837,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     {
       const int nvec = P.d * 2 / 16;
       dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
-      moe::combine_kernel<bf16><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+      launch_pdl(moe::combine_kernel<bf16>, grid, 256, 0, st, yrows, ys, slot, T, P.k, P.d,
                                                       static_cast<bf16*>(y), P.rows_max);
     }
     tm.at(13);
@@ -838,7 +865,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     dim3 grid((nmax + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
     tm.at(8);
-    moe::simt_gemm_kernel<float, float, float, moe::EPI_SWIGLU><<<grid, 256, 0, st>>>(a, b);
+    launch_pdl(moe::simt_gemm_kernel<float, float, float, moe::EPI_SWIGLU>, grid, 256, 0, st, a, b);
     tm.at(9);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
   }
@@ -850,7 +877,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
     dim3 grid((P.d + moe::SG_BN - 1) / moe::SG_BN,
               static_cast<unsigned>((gy + moe::SG_BM - 1) / moe::SG_BM), P.ds ? 2 : 1);
     tm.at(10);
-    moe::simt_gemm_kernel<float, float, float, moe::EPI_SCALE><<<grid, 256, 0, st>>>(a, b);
+    launch_pdl(moe::simt_gemm_kernel<float, float, float, moe::EPI_SCALE>, grid, 256, 0, st, a, b);
     tm.at(11);
     if (launched() != MOE_OK) return MOE_ERR_CUDA;
   }
@@ -858,7 +885,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
   {
     const int nvec = P.d * 4 / 16;
     dim3 grid((T + 7) / 8, (nvec + moe::PERMUTE_CHUNK_VECS - 1) / moe::PERMUTE_CHUNK_VECS);
-    moe::combine_kernel<float><<<grid, 256, 0, st>>>(yrows, ys, slot, T, P.k, P.d,
+    launch_pdl(moe::combine_kernel<float>, grid, 256, 0, st, yrows, ys, slot, T, P.k, P.d,
                                                      static_cast<float*>(y), P.rows_max);
   }
   tm.at(13);

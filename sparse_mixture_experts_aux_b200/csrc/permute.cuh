@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(
     const int32_t* __restrict__ tile_start, int32_t* __restrict__ slot_pos,
     float* __restrict__ row_gate, TX* __restrict__ xp, int64_t rows_max,
     const float* __restrict__ scale_in = nullptr, float* __restrict__ scale_out = nullptr) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;  // warp-uniform
@@ -100,6 +102,8 @@ template <typename TY>
 __global__ void __launch_bounds__(256) combine_kernel(
     const TY* __restrict__ yrows, const TY* __restrict__ ys, const int32_t* __restrict__ slot_pos,
     int T, int k, int d, TY* __restrict__ y, int64_t rows_max) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int VN = Vec16<TY>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;

@@ -60,6 +60,8 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
 // the rounding error of a long dot product well below one sequential chain.
 template <typename TA, typename TB, typename TC, int EPI>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGroup g0, SimtGroup g1) {
+  pdl_wait();
+  pdl_launch_dependents();
   const SimtGroup g = blockIdx.z == 0 ? g0 : g1;
   if (!g.active) return;
   const int k_len = g.K;
@@ -212,6 +214,8 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const TA* __restric
                                                              const float* __restrict__ W_r,
                                                              int T, int K, int E, int splits,
                                                              float* __restrict__ logits) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ __align__(16) float As[RW_BK][RW_BM + 4];
   __shared__ __align__(16) float Bs[RW_BK][RW_BN + 4];
   const int k_len = K / splits;
@@ -330,6 +334,8 @@ __global__ void __launch_bounds__(256) router_narrow_kernel(const TA* __restrict
                                                             const float* __restrict__ W_r, int T,
                                                             int d, int E, int splits,
                                                             float* __restrict__ logits) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int TOK = NarrowShape<NE>::TOK;
   constexpr int TB = NarrowShape<NE>::TB;
   __shared__ __align__(16) float ws[NE][NARROW_KC];
@@ -423,6 +429,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 constexpr int ROUTE_TOK_PER_WARP = ROUTE_CHUNK / ROUTE_WARPS;
+constexpr int ROUTE_FAST_SPLITS = 16;  // K-split partials loaded together (few experts)
 constexpr int ROUTE_RANK_GROUPS = ROUTE_CHUNK / 32;
 static_assert(ROUTE_CHUNK % 32 == 0 && ROUTE_RANK_GROUPS <= ROUTE_WARPS, "route chunk shape");
 
@@ -433,12 +440,124 @@ __host__ __device__ constexpr size_t route_smem_bytes(int E) {
 
 enum { GATE_RENORM = 0, GATE_RAW = 1, GATE_SIGMOID = 2 };
 
+// ---------------------------------------------------------------------------
+// Scan over experts (one block, thread e = expert e, E <= nthreads, nthreads a
+// power of two <= 1024):
+//   base[b][e]   = assignments to e in chunks before b (stable token-order rank base)
+//   counts[e]    = routed assignments to e (before the capacity cut)
+//   kept_e       = min(counts[e], C); segment of ceil(kept_e / ROW_TILE) tiles
+//   tile_start   = exclusive scan of the segment sizes; tile_start[E] = total
+//   pair_start   = exclusive scan of ceil(segment tiles / 2) (CTA-pair tiles)
+//   probsum[e]   = sum of the probability partials, fp64, fixed order
+//   aux          = E * sum_e (counts_e / (T k)) (probsum_e / T), fp64, fixed tree
+// and clears the call's status word. s_scan holds 2 * nthreads ints, s_sum
+// nthreads doubles. Every thread of the block must call it.
+// ---------------------------------------------------------------------------
+__device__ void scan_experts(int nthreads, const int32_t* __restrict__ hist, int nblk,
+                             const double* __restrict__ psum_part, int nparts, int E, int64_t T,
+                             int k, int64_t C, int32_t* __restrict__ counts,
+                             int32_t* __restrict__ base, int32_t* __restrict__ tile_start,
+                             int32_t* __restrict__ pair_start, double* __restrict__ probsum,
+                             float* __restrict__ aux, int* __restrict__ call_err, int64_t rows_max,
+                             int* s_scan, double* s_sum) {
+  const int e = threadIdx.x;
+  if (e == 0 && call_err != nullptr) *call_err = 0;  // the GEMMs of this call run after this
+  int tiles = 0;
+  double term = 0.0;
+  if (e < E) {
+    int run = 0;
+#pragma unroll 8
+    for (int b = 0; b < nblk; ++b) {
+      base[(size_t)b * E + e] = run;
+      run += hist[(size_t)b * E + e];
+    }
+    counts[e] = run;
+    const int kept = (C >= 0 && (int64_t)run > C) ? (int)C : run;
+    tiles = (kept + ROW_TILE - 1) / ROW_TILE;
+    double ps = 0.0;
+#pragma unroll 8
+    for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
+    probsum[e] = ps;
+    term = (double)run * ps;
+  }
+  if (e < nthreads) {
+    s_scan[e] = tiles;
+    s_sum[e] = term;
+  }
+  __syncthreads();
+  int cur = 0;
+  for (int off = 1; off < nthreads; off <<= 1) {  // inclusive Hillis-Steele scan
+    if (e < nthreads) {
+      const int v = s_scan[cur * nthreads + e] + (e >= off ? s_scan[cur * nthreads + e - off] : 0);
+      s_scan[(cur ^ 1) * nthreads + e] = v;
+    }
+    cur ^= 1;
+    __syncthreads();
+  }
+  if (e < E) tile_start[e] = s_scan[cur * nthreads + e] - tiles;
+  if (e == E - 1) {
+    tile_start[E] = s_scan[cur * nthreads + e];
+#if defined(MOE_DEBUG)
+    if ((int64_t)s_scan[cur * nthreads + e] * ROW_TILE > rows_max) flag_bounds();
+#else
+    (void)rows_max;
+#endif
+  }
+  // the same scan over pairs of tiles (a CTA pair computes two tiles of one expert)
+  const int pairs = (tiles + 1) / 2;
+  __syncthreads();
+  if (e < nthreads) s_scan[e] = pairs;
+  cur = 0;
+  __syncthreads();
+  for (int off = 1; off < nthreads; off <<= 1) {
+    if (e < nthreads) {
+      const int v = s_scan[cur * nthreads + e] + (e >= off ? s_scan[cur * nthreads + e - off] : 0);
+      s_scan[(cur ^ 1) * nthreads + e] = v;
+    }
+    cur ^= 1;
+    __syncthreads();
+  }
+  if (e < E) pair_start[e] = s_scan[cur * nthreads + e] - pairs;
+  if (e == E - 1) pair_start[E] = s_scan[cur * nthreads + e];
+  for (int half = nthreads / 2; half > 0; half >>= 1) {  // fixed-shape tree sum
+    if (e < half) s_sum[e] += s_sum[e + half];
+    __syncthreads();
+  }
+  if (e == 0) {
+    const double denom = (double)T * (double)k * (double)T;
+    aux[0] = (T > 0) ? (float)((double)E * s_sum[0] / denom) : 0.f;
+  }
+}
+
+// Threads of the scan for E experts.
+__host__ __device__ inline int scan_threads(int E) {
+  int n = 32;
+  while (n < E) n <<= 1;
+  return n;
+}
+
+// Arguments of the scan when the routing kernel runs it itself (one chunk).
+struct ScanArgs {
+  bool fused;
+  int64_t C, rows_max;
+  int32_t* counts;
+  int32_t* base;
+  int32_t* tile_start;
+  int32_t* pair_start;
+  double* probsum;
+  float* aux;
+  int* call_err;
+};
+
 template <int NV>
 __global__ void __launch_bounds__(256, 1) route_kernel(
     float* __restrict__ logits, int splits, const float* __restrict__ bias,
     const float* __restrict__ sel_bias, int gate_mode, int n_group, int topk_group, int T, int E,
     int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-    int32_t* __restrict__ lrank_out, int32_t* __restrict__ hist, double* __restrict__ psum_part) {
+    int32_t* __restrict__ lrank_out, int32_t* __restrict__ hist, double* __restrict__ psum_part,
+    const ScanArgs sa) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t route_smem_raw[];
   double* red = reinterpret_cast<double*>(route_smem_raw);  // [ROUTE_WARPS][E]
   uint32_t* bm = reinterpret_cast<uint32_t*>(red + (size_t)ROUTE_WARPS * E);  // [groups][E]
@@ -447,7 +566,9 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
   const int blk = blockIdx.x;
   for (int i = threadIdx.x; i < ROUTE_RANK_GROUPS * E; i += blockDim.x) bm[i] = 0u;
 
-  const int t_warp0 = blk * ROUTE_CHUNK + warp * ROUTE_TOK_PER_WARP;
+  // Warp w takes the chunk's tokens w, w + 8, w + 16, ... (interleaved, so that
+  // a short batch still keeps every warp busy).
+  auto tok = [&](int j) { return blk * ROUTE_CHUNK + j * ROUTE_WARPS + warp; };
   const bool grouped = n_group > 1 && topk_group < n_group;
   const int gsize = grouped ? E / n_group : E;
   double ps[NV];
@@ -461,11 +582,32 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
   }
 
   // The next token's logits are loaded (and their K-split partials summed, in
-  // a fixed order) while the current token is processed.
+  // a fixed order) while the current token is processed. For few experts all
+  // of a logit's partials are loaded before any is added, so the loads are in
+  // flight together instead of one round trip after another.
   const size_t split_stride = (size_t)T * E;
   float nxt[NV];
   auto load_logits = [&](int t) {
     const float* row = logits + (size_t)t * E;
+    if (NV <= 2 && splits <= ROUTE_FAST_SPLITS) {
+      float part[NV][ROUTE_FAST_SPLITS];
+#pragma unroll
+      for (int sp = 0; sp < ROUTE_FAST_SPLITS; ++sp)
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const int e = lane + 32 * i;
+          part[i][sp] = (sp < splits && e < E) ? row[sp * split_stride + e] : 0.f;
+        }
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        float r = part[i][0];
+#pragma unroll
+        for (int sp = 1; sp < ROUTE_FAST_SPLITS; ++sp)
+          if (sp < splits) r += part[i][sp];
+        nxt[i] = r;
+      }
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
@@ -477,14 +619,14 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
       nxt[i] = r;
     }
   };
-  if (t_warp0 < T) load_logits(t_warp0);
+  if (tok(0) < T) load_logits(tok(0));
   for (int j = 0; j < ROUTE_TOK_PER_WARP; ++j) {
-    const int t = t_warp0 + j;
+    const int t = tok(j);
     if (t >= T) break;  // warp-uniform
     float raw[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) raw[i] = nxt[i];
-    if (j + 1 < ROUTE_TOK_PER_WARP && t + 1 < T) load_logits(t + 1);
+    if (j + 1 < ROUTE_TOK_PER_WARP && tok(j + 1) < T) load_logits(tok(j + 1));
     float* row = logits + (size_t)t * E;
     float v[NV];
     uint32_t removed = 0u;
@@ -648,86 +790,33 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
       lrank_out[(size_t)t * k + sl] = wbase[warp * E + e] + __popc(bm[warp * E + e] & lt);
     }
   }
+  if (sa.fused) {
+    // a batch of one chunk (E <= 256): the scan runs here, on this chunk's
+    // histogram and probability sums, instead of in a kernel of its own
+    __shared__ int f_scan[2 * 256];
+    __shared__ double f_sum[256];
+    __syncthreads();  // hist and psum_part are written (block-visible)
+    scan_experts(scan_threads(E), hist, 1, psum_part, 1, E, T, k, sa.C, sa.counts, sa.base,
+                 sa.tile_start, sa.pair_start, sa.probsum, sa.aux, sa.call_err, sa.rows_max,
+                 f_scan, f_sum);
+  }
 }
 
-// ---------------------------------------------------------------------------
-// Scan (one block of 1024 threads, thread e = expert e):
-//   base[b][e]   = assignments to e in chunks before b (stable token-order rank base)
-//   counts[e]    = routed assignments to e (before the capacity cut)
-//   kept_e       = min(counts[e], C); segment of ceil(kept_e / ROW_TILE) tiles
-//   tile_start   = exclusive scan of the segment sizes; tile_start[E] = total
-//   pair_start   = exclusive scan of ceil(segment tiles / 2) (CTA-pair tiles)
-//   probsum[e]   = sum of the probability partials, fp64, fixed order
-//   aux          = E * sum_e (counts_e / (T k)) (probsum_e / T), fp64, fixed tree
-// and clears the call's status word.
-// ---------------------------------------------------------------------------
+// The scan as its own kernel: one block of nthreads = the smallest power of two
+// >= max(E, 32) threads.
 __global__ void __launch_bounds__(1024) scan_kernel(
     const int32_t* __restrict__ hist, int nblk, const double* __restrict__ psum_part, int nparts,
     int E, int64_t T, int k, int64_t C, int32_t* __restrict__ counts, int32_t* __restrict__ base,
     int32_t* __restrict__ tile_start, int32_t* __restrict__ pair_start,
     double* __restrict__ probsum, float* __restrict__ aux, int* __restrict__ call_err,
     int64_t rows_max) {
-  __shared__ int s_scan[2][1024];
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ int s_scan[2 * 1024];
   __shared__ double s_sum[1024];
-  const int e = threadIdx.x;
-  if (e == 0 && call_err != nullptr) *call_err = 0;  // the GEMMs of this call run after this
-  int tiles = 0;
-  double term = 0.0;
-  if (e < E) {
-    int run = 0;
-#pragma unroll 8
-    for (int b = 0; b < nblk; ++b) {
-      base[(size_t)b * E + e] = run;
-      run += hist[(size_t)b * E + e];
-    }
-    counts[e] = run;
-    const int kept = (C >= 0 && (int64_t)run > C) ? (int)C : run;
-    tiles = (kept + ROW_TILE - 1) / ROW_TILE;
-    double ps = 0.0;
-#pragma unroll 8
-    for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
-    probsum[e] = ps;
-    term = (double)run * ps;
-  }
-  s_scan[0][e] = tiles;
-  s_sum[e] = term;
-  __syncthreads();
-  int cur = 0;
-  for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = s_scan[cur][e] + (e >= off ? s_scan[cur][e - off] : 0);
-    s_scan[cur ^ 1][e] = v;
-    cur ^= 1;
-    __syncthreads();
-  }
-  if (e < E) tile_start[e] = s_scan[cur][e] - tiles;
-  if (e == E - 1) {
-    tile_start[E] = s_scan[cur][e];
-#if defined(MOE_DEBUG)
-    if ((int64_t)s_scan[cur][e] * ROW_TILE > rows_max) flag_bounds();  // segments overflow
-#endif
-  }
-  // the same scan over pairs of tiles (a CTA pair computes two tiles of one expert)
-  const int pairs = (tiles + 1) / 2;
-  __syncthreads();
-  s_scan[0][e] = pairs;
-  cur = 0;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int v = s_scan[cur][e] + (e >= off ? s_scan[cur][e - off] : 0);
-    s_scan[cur ^ 1][e] = v;
-    cur ^= 1;
-    __syncthreads();
-  }
-  if (e < E) pair_start[e] = s_scan[cur][e] - pairs;
-  if (e == E - 1) pair_start[E] = s_scan[cur][e];
-  for (int half = 512; half > 0; half >>= 1) {  // fixed-shape tree sum
-    if (e < half) s_sum[e] += s_sum[e + half];
-    __syncthreads();
-  }
-  if (e == 0) {
-    const double denom = (double)T * (double)k * (double)T;
-    aux[0] = (T > 0) ? (float)((double)E * s_sum[0] / denom) : 0.f;
-  }
+  scan_experts(blockDim.x, hist, nblk, psum_part, nparts, E, T, k, C, counts, base, tile_start,
+               pair_start, probsum, aux, call_err, rows_max, s_scan, s_sum);
 }
+
 
 }  // namespace moe

@@ -61,6 +61,8 @@ struct RtcMaps {
 __global__ void __launch_bounds__(256) split_router_weights_kernel(const float* __restrict__ w,
                                                                    int64_t n,
                                                                    __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const float v = w[i];
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc::tmem_alloc(tc::smem_addr(tmem_slot), TMEM_COLS);
     tc::tmem_relinquish();
   }
+  pdl_wait();
+  pdl_launch_dependents();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();

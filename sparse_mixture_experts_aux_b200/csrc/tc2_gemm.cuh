@@ -260,12 +260,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t peer_abort = mapa_shared(tc::smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u);
 
   const Tc2Group& G0 = p.g[0];
-  if (G0.tile_start != nullptr) {
-    for (int i = threadIdx.x; i <= G0.E; i += NUM_THREADS) {
-      s_ts[i] = G0.tile_start[i];
-      s_ps[i] = G0.pair_start[i];
-    }
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(full_bar(s), 1);
@@ -282,6 +276,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tmem_alloc_pair(tc::smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish_pair();
+  }
+  pdl_wait();  // the routing results and rows this GEMM reads are complete
+  pdl_launch_dependents();
+  if (G0.tile_start != nullptr) {
+    for (int i = threadIdx.x; i <= G0.E; i += NUM_THREADS) {
+      s_ts[i] = G0.tile_start[i];
+      s_ps[i] = G0.pair_start[i];
+    }
   }
   tc::tc_fence_before();
   __syncthreads();

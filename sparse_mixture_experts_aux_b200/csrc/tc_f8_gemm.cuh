@@ -258,6 +258,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc::tmem_alloc(tc::smem_addr(tmem_slot), TMEM_COLS);
     tc::tmem_relinquish();
   }
+  pdl_wait();  // the routing results and rows this GEMM reads are complete
+  pdl_launch_dependents();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -598,6 +600,8 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(
     const TW* __restrict__ w, int64_t rows, int cols, uint8_t* __restrict__ codes,
     float* __restrict__ scales, const int32_t* __restrict__ tile_start = nullptr,
     const int32_t* __restrict__ counts = nullptr, int E = 0, int64_t C = -1) {
+  pdl_wait();
+  pdl_launch_dependents();
   // Rows of the permuted buffers (tile_start given): only the rows an expert
   // actually holds (min(count, C) at the head of its 128-row segments) are
   // quantised; the padding rows behind them are left alone.

@@ -379,8 +379,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
 
   const TcGroup& G0 = p.g[0];
-  if (G0.tile_start != nullptr)
-    for (int i = threadIdx.x; i <= G0.E; i += NUM_THREADS) s_ts[i] = G0.tile_start[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
@@ -398,6 +396,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // the routing results and rows this GEMM reads are complete
+  pdl_launch_dependents();
+  if (G0.tile_start != nullptr)
+    for (int i = threadIdx.x; i <= G0.E; i += NUM_THREADS) s_ts[i] = G0.tile_start[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -75,7 +75,7 @@ def test_dequantizer_every_code_bit_exact():
     # rows of all 16 codes (twice) in blocks whose exponents lie within 23 of the
     # row's largest: the layer's decode is exact there
     codes = np.resize(np.arange(16, dtype=np.uint8), (6, 32 * 4))
-    exps = np.array([[0, -5, -23, 3], [7, 7, 7, 7], [-40, -44, -63, -50],
+    exps = np.array([[0, -5, -23, -1], [7, 7, 7, 7], [-40, -44, -63, -50],
                      [20, 0, 12, 1], [0, 0, 0, 0], [-1, -2, -3, -4]], dtype=np.int64)
     rf = row_factors_of(codes, exps)
     packed = torch.from_numpy(pack_e2m1(codes)).cuda()
