@@ -41,6 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, weights) -> DRAM bytes / algorithmic bytes of the gate/up kernel, from one ncu
 # capture of that kernel as built (profiles/); absent = not captured for the current build.
 TRAFFIC_RATIO = {("mixtral", "dtype"): 539.386880 / 545.259520}
+# the same for the down kernel (CTA pairs), T=1024 E=2 case: DRAM 344.265 MB / 310.4 MB
+DOWN_TRAFFIC_RATIO = {("mixtral", "dtype"): 344.265216 / 310.378496}
 
 
 def parse_args(argv=None):
@@ -404,6 +406,8 @@ def run_ours(args, rank, world, local_rank):
                             if traffic_ratio is not None else None)
     rl = {"kernel": KERNEL_NAMES[4], **rl}
     rl_down = kernel_roofline(wk["flops_down"], wk["bytes_down"], k_down, tensor_peak, hbm_peak)
+    down_ratio = DOWN_TRAFFIC_RATIO.get((args.workload, args.weights))
+    rl_down["traffic"] = down_ratio * wk["bytes_down"] if down_ratio is not None else None
     roof_ms = max(wk["flops"] / (tensor_peak * 1e12),
                   (wk["w_bytes"] + wk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
     roof_ms_sust = max(wk["flops"] / (tensor_sust * 1e12),
