@@ -16,6 +16,7 @@
 #include "tc2_gemm.cuh"
 #include "tc_f8_gemm.cuh"
 #include "router_tc.cuh"
+#include "tc_wq_swap.cuh"
 
 namespace {
 
@@ -244,6 +245,30 @@ void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
     launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 128, WQ>, grid, NUM_THREADS, F8Shape<128, WQ>::SMEM_BYTES, st, maps, fp);
 }
 
+// Quantised-weight grouped GEMM for at most 64 tokens (operands swapped,
+// decoded weights in TMEM) with token boxes of `nb` rows (32 or 64).
+template <int EPI, int WQ>
+bool wq_attr() {
+  return cudaFuncSetAttribute(moe::wqs::tc_wq_swap_kernel<EPI, 32, WQ>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moe::wqs::WqShape<32, WQ>::SMEM_BYTES) == cudaSuccess &&
+         cudaFuncSetAttribute(moe::wqs::tc_wq_swap_kernel<EPI, 64, WQ>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moe::wqs::WqShape<64, WQ>::SMEM_BYTES) == cudaSuccess;
+}
+
+template <int EPI, int WQ>
+void launch_wq(int nb, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
+               const moe::wqs::WqParams& wp) {
+  using namespace moe::wqs;
+  if (nb == 32)
+    launch_pdl(tc_wq_swap_kernel<EPI, 32, WQ>, grid, NUM_THREADS, WqShape<32, WQ>::SMEM_BYTES, st,
+               maps, wp);
+  else
+    launch_pdl(tc_wq_swap_kernel<EPI, 64, WQ>, grid, NUM_THREADS, WqShape<64, WQ>::SMEM_BYTES, st,
+               maps, wp);
+}
+
 // 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32);
 // Q8: E4M3 operands.
 template <int EPI, bool Q8 = false>
@@ -320,11 +345,16 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 32, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32, true>())
       return MOE_ERR_CUDA;
     if (!f8_attrs<moe::tcf8::WQ_FP8>() || !f8_attrs<moe::tcf8::WQ_MXFP4>()) return MOE_ERR_CUDA;
+    if (!wq_attr<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_FP8>() ||
+        !wq_attr<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>() ||
+        !wq_attr<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>() ||
+        !wq_attr<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_MXFP4>())
+      return MOE_ERR_CUDA;
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
         !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(moe::rtc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             moe::rtc::SMEM_BYTES) != cudaSuccess)
+                             moe::rtc::SMEM_LIMIT) != cudaSuccess)
       return MOE_ERR_CUDA;
     const int rs = static_cast<int>(moe::route_smem_bytes(moe::tc::MAX_E));
     if (cudaFuncSetAttribute(moe::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -453,7 +483,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
     rp.call_err = reinterpret_cast<int*>(ws + P.o_status);
     dim3 grid((T + moe::rtc::BM - 1) / moe::rtc::BM, (P.E + P.router_n - 1) / P.router_n,
               P.router_split);
-    launch_pdl(moe::rtc::router_tc_kernel, grid, moe::rtc::NUM_THREADS, moe::rtc::SMEM_BYTES, st, maps,
+    launch_pdl(moe::rtc::router_tc_kernel, grid, moe::rtc::NUM_THREADS, moe::rtc::smem_bytes(P.router_n), st, maps,
                                                                                           rp);
   } else if (P.router_narrow) {
     if (P.E <= 8) {
@@ -656,8 +686,69 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     } else if (dims->weight_format == MOE_WEIGHTS_FP8 || dims->weight_format == MOE_WEIGHTS_MXFP4) {
       // FP8 or MXFP4 expert weights: 1-CTA kernels that dequantise the weight
-      // tiles on chip
+      // tiles on chip; at most 64 tokens: operands swapped, decoded weights in TMEM
       const bool mx = dims->weight_format == MOE_WEIGHTS_MXFP4;
+      if (P.T <= 64) {
+        const int nb = P.T <= 32 ? 32 : 64;
+        const float* sc = dims->weight_scales;
+        const size_t gsz = static_cast<size_t>(E) * P.de;
+        const int cpb = mx ? 2 : 1;  // codes per byte
+        moe::tc::TcMaps up, dn;
+        memset(&up, 0, sizeof(up));
+        memset(&dn, 0, sizeof(dn));
+        const bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, nb, 2) &&
+                        encode_map_u8(&up.b0[0], W_g, P.d / cpb, P.de, E, moe::tc::BM) &&
+                        encode_map_u8(&up.b1[0], W_u, P.d / cpb, P.de, E, moe::tc::BM) &&
+                        encode_map(&dn.a[0], h, P.de, P.rows_max, 1, nb, 2) &&
+                        encode_map_u8(&dn.b0[0], W_d, P.de / cpb, P.d, E, moe::tc::BM);
+        if (!ok) return MOE_ERR_CUDA;
+        const uint8_t* bs = dims->weight_block_scales;
+        const size_t gbs = gsz * (P.d / 32);
+        moe::wqs::WqParams wu{}, wd{};
+        wu.timeout_ns = wd.timeout_ns = wait_tmo;
+        wu.drain_timeout_ns = wd.drain_timeout_ns = kDrainTimeoutNs;
+        wu.call_err = wd.call_err = call_err;
+        wu.grp.tile_start = wd.grp.tile_start = tile_start;
+        wu.grp.E = wd.grp.E = E;
+        wu.grp.rows = wd.grp.rows = rows_cap;
+        wu.grp.n_tiles = (P.de + moe::tc::BM - 1) / moe::tc::BM;
+        wu.grp.k_blocks = P.d / moe::tc::BK;
+        wu.grp.N = P.de;
+        wu.grp.out = h;
+        wu.grp.scale0 = sc;
+        wu.grp.scale1 = sc + gsz;
+        wu.grp.scale_stride = P.de;
+        wd.grp.n_tiles = (P.d + 2 * moe::tc::BM - 1) / (2 * moe::tc::BM);
+        wd.grp.k_blocks = P.de / moe::tc::BK;
+        wd.grp.N = P.d;
+        wd.grp.out = yrows;
+        wd.grp.row_gate = rowgate;
+        wd.grp.scale0 = wd.grp.scale1 = sc + 2 * gsz;
+        wd.grp.scale_stride = P.d;
+        if (mx) {
+          wu.grp.bscale0 = bs;
+          wu.grp.bscale1 = bs + gbs;
+          wu.grp.bscale_stride = static_cast<int64_t>(P.de) * (P.d / 32);
+          wu.grp.kblk = P.d / 32;
+          wd.grp.bscale0 = wd.grp.bscale1 = bs + 2 * gbs;
+          wd.grp.bscale_stride = static_cast<int64_t>(P.d) * (P.de / 32);
+          wd.grp.kblk = P.de / 32;
+        }
+        tm.at(8);
+        if (mx)
+          launch_wq<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>(nb, num_sms, st, up, wu);
+        else
+          launch_wq<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_FP8>(nb, num_sms, st, up, wu);
+        tm.at(9);
+        if (launched() != MOE_OK) return MOE_ERR_CUDA;
+        tm.at(10);
+        if (mx)
+          launch_wq<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_MXFP4>(nb, num_sms, st, dn, wd);
+        else
+          launch_wq<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>(nb, num_sms, st, dn, wd);
+        tm.at(11);
+        if (launched() != MOE_OK) return MOE_ERR_CUDA;
+      } else {
       const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
       const float* sc = dims->weight_scales;
       const size_t gsz = static_cast<size_t>(E) * P.de;
@@ -719,6 +810,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         launch_f8<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>(arows, num_sms, st, dn, fd);
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
+      }  // more than 64 tokens
     } else {
     // (4) gate/up projection + SwiGLU, (5) down projection scaled by the gates.
     // CTA-pair tiles (256 rows) cut the operand traffic per SM by a third but

@@ -17,7 +17,8 @@
 // Tile: 128 tokens x N experts (N = E rounded up to 16, at most 128) over one
 // K range (grid.z splits K; the routing kernel sums the split partials in a
 // fixed order). Stage: the x box (128 x 64 bf16) and the three terms' boxes
-// (N x 64 each), all TMA with the 128-byte swizzle. Warp 0 = TMA producer,
+// (N x 64 each), all TMA with the 128-byte swizzle; as many stages as fit
+// (3 at N = 128, 8 at small N), with x's boxes prefetched into L2 ahead. Warp 0 = TMA producer,
 // warp 1 = TMEM owner and MMA issuer, warps 2..9 = epilogue (two per TMEM lane
 // quadrant, each summing half of the N columns in registers). TMEM holds two
 // 128 x N accumulators, so one chunk is summed while the next is computed.
@@ -32,17 +33,29 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int MAX_N = 128;
 constexpr int KC = 2;  // K blocks (64 deep) per accumulation chunk
-constexpr int STAGES = 3;
+constexpr int MAX_STAGES = 8;
+constexpr int X_PREFETCH = 8;  // K blocks of x prefetched into L2 ahead of their loads
 constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = MAX_N * BK * 2;          // one term's box at the largest N
-constexpr int STAGE_BYTES = A_BYTES + 3 * B_BYTES;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr int SMEM_LIMIT = 232448;
 constexpr uint32_t TMEM_COLS = 256;  // two accumulators of up to 128 columns
-static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned boxes");
+static_assert(A_BYTES % 1024 == 0, "1024-byte aligned boxes");
+
+// Stage geometry for tiles of N experts: the x box and the three terms' N-row
+// boxes, as many stages as fit (at most MAX_STAGES): 3 at N = 128, 8 at N = 16.
+__host__ __device__ constexpr int stage_bytes(int N) { return A_BYTES + 3 * N * BK * 2; }
+__host__ __device__ constexpr int stages_for(int N) {
+  return (SMEM_LIMIT - 1024 - BAR_BYTES) / stage_bytes(N) < MAX_STAGES
+             ? (SMEM_LIMIT - 1024 - BAR_BYTES) / stage_bytes(N)
+             : MAX_STAGES;
+}
+__host__ __device__ constexpr int smem_bytes(int N) {
+  return 1024 + stages_for(N) * stage_bytes(N) + BAR_BYTES;
+}
+static_assert(smem_bytes(MAX_N) <= SMEM_LIMIT && smem_bytes(16) <= SMEM_LIMIT, "shared memory");
+static_assert(stages_for(MAX_N) >= 2, "at least double buffering");
 
 struct RtcParams {
   int T, E, N;          // tokens, experts, columns of one tile (multiple of 16, <= MAX_N)
@@ -51,6 +64,14 @@ struct RtcParams {
   unsigned long long timeout_ns, drain_timeout_ns;
   int* call_err;
 };
+
+// Prefetch a tiled box of a tensor map into L2 (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
 
 struct RtcMaps {
   CUtensorMap x;  // bf16 [T][d], box {64, 128}
@@ -79,6 +100,9 @@ __global__ void __launch_bounds__(256) split_router_weights_kernel(const float* 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     router_tc_kernel(const __grid_constant__ RtcMaps maps, const RtcParams p) {
   extern __shared__ uint8_t smem_raw[];
+  const int STAGES = stages_for(p.N);
+  const int STAGE_BYTES = stage_bytes(p.N);
+  const uint32_t b_bytes = (uint32_t)p.N * BK * 2;  // one term's box
   const uint32_t raw_addr = tc::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -124,7 +148,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int kb0 = blockIdx.z * p.k_blocks;
   const int nkb = p.k_blocks;
   const int nch = (nkb + KC - 1) / KC;
-  const uint32_t b_bytes = (uint32_t)p.N * BK * 2;
   const unsigned long long tmo = p.timeout_ns, drain_tmo = p.drain_timeout_ns;
 
   if (warp == 0) {
@@ -132,6 +155,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       tc::prefetch_map(&maps.x);
       tc::prefetch_map(&maps.w);
+      // x streams from HBM once per N tile: its boxes are prefetched into L2
+      // X_PREFETCH blocks ahead, so the ring's loads see L2 latency
+      for (int kb = 0; kb < X_PREFETCH && kb < nkb; ++kb)
+        tma_prefetch_l2_2d(&maps.x, (kb0 + kb) * BK, m0);
       uint32_t issued = 0, last_par = 0;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -145,7 +172,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc::tma_load_2d(sa, &maps.x, fb, kx, m0);
 #pragma unroll
         for (int t = 0; t < 3; ++t)
-          tc::tma_load_3d(sa + A_BYTES + t * B_BYTES, &maps.w, fb, kx, n0, t);
+          tc::tma_load_3d(sa + A_BYTES + t * b_bytes, &maps.w, fb, kx, n0, t);
+        if (kb + X_PREFETCH < nkb) tma_prefetch_l2_2d(&maps.x, kx + X_PREFETCH * BK, m0);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
       }
@@ -177,7 +205,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the smallest term first; a fresh accumulator at the chunk's first MMA
 #pragma unroll
           for (int t = 2; t >= 0; --t) {
-            const uint64_t bd = tc::sw128_kmajor_desc(sa + A_BYTES + t * B_BYTES);
+            const uint64_t bd = tc::sw128_kmajor_desc(sa + A_BYTES + t * b_bytes);
 #pragma unroll
             for (int kk = 0; kk < BK / tc::UMMA_K; ++kk)
               tc::tc_mma(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc,
