@@ -18,7 +18,7 @@
 // K range (grid.z splits K; the routing kernel sums the split partials in a
 // fixed order). Stage: the x box (128 x 64 bf16) and the three terms' boxes
 // (N x 64 each), all TMA with the 128-byte swizzle; as many stages as fit
-// (3 at N = 128, 8 at small N), with x's boxes prefetched into L2 ahead. Warp 0 = TMA producer,
+// (3 at N = 128, 8 at small N). Warp 0 = TMA producer,
 // warp 1 = TMEM owner and MMA issuer, warps 2..9 = epilogue (two per TMEM lane
 // quadrant, each summing half of the N columns in registers). TMEM holds two
 // 128 x N accumulators, so one chunk is summed while the next is computed.
@@ -34,7 +34,6 @@ constexpr int BK = 64;
 constexpr int MAX_N = 128;
 constexpr int KC = 2;  // K blocks (64 deep) per accumulation chunk
 constexpr int MAX_STAGES = 8;
-constexpr int X_PREFETCH = 8;  // K blocks of x prefetched into L2 ahead of their loads
 constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;
 constexpr int A_BYTES = BM * BK * 2;
@@ -65,13 +64,6 @@ struct RtcParams {
   int* call_err;
 };
 
-// Prefetch a tiled box of a tensor map into L2 (no shared memory involved).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
 
 struct RtcMaps {
   CUtensorMap x;  // bf16 [T][d], box {64, 128}
@@ -155,10 +147,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       tc::prefetch_map(&maps.x);
       tc::prefetch_map(&maps.w);
-      // x streams from HBM once per N tile: its boxes are prefetched into L2
-      // X_PREFETCH blocks ahead, so the ring's loads see L2 latency
-      for (int kb = 0; kb < X_PREFETCH && kb < nkb; ++kb)
-        tma_prefetch_l2_2d(&maps.x, (kb0 + kb) * BK, m0);
       uint32_t issued = 0, last_par = 0;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -173,7 +161,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 3; ++t)
           tc::tma_load_3d(sa + A_BYTES + t * b_bytes, &maps.w, fb, kx, n0, t);
-        if (kb + X_PREFETCH < nkb) tma_prefetch_l2_2d(&maps.x, kx + X_PREFETCH * BK, m0);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
       }

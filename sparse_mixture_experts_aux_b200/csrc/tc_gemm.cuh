@@ -154,6 +154,13 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// The same with the first test inline: a phase that has already completed
+// costs one try_wait instead of a call (the bounded loop stays out of line).
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long timeout_ns) {
+  return mbar_try_wait(bar, parity) || wait_bounded(bar, parity, abort_flag, timeout_ns);
+}
+
 // Same, not stopping on the abort flag (it raises it when it gives up): used
 // only in teardown, to let copies and MMAs already in flight land before
 // shared memory and TMEM are released.

@@ -24,15 +24,17 @@
 // gate_c (d s_d) as bf16, s_* the per-row weight scale (FP8) or row factor
 // (MXFP4).
 //
-// Warp roles (480 threads): 0 activation producer, 1 TMEM owner and MMA issuer,
-// 2..5 epilogue (TMEM lane quadrant w % 4), 6..13 converters (matrix
-// (w - 6) / 4, lane quadrant w % 4), 14 weight-code producer.
+// Warp roles (512 threads): 0 activation producer, 1 TMEM owner and MMA issuer
+// of matrix 0, 2..5 epilogue (TMEM lane quadrant w % 4), 6..13 converters
+// (matrix (w - 6) / 4, lane quadrant w % 4), 14 weight-code producer, 15 MMA
+// issuer of matrix 1.
 // Synchronisation, all waits bounded:
 //   qfull[q]  code producer expect_tx + TMA bytes;     qempty[q] 8 converter warps
-//   bfull[b]  activation producer expect_tx + bytes;   bempty[b] MMA commit
+//   bfull[b]  activation producer expect_tx + bytes (waited by the first
+//             converter warp);                          bempty[b] 2 MMA commits
 //   afull[a]  8 converter warps (after tcgen05.st, wait::st and the tcgen05
-//             fence);                                   aempty[a] MMA commit
-//   tfull[2]  MMA commit;                               tempty[2] 4 epilogue warps
+//             fence);                                   aempty[a] 2 MMA commits
+//   tfull[2]  2 MMA commits;                            tempty[2] 4 epilogue warps
 // Sources: AI Engineering Illustrated "Mixture of Experts", "Trade-offs to
 // weigh" (small-batch MoE is bound by reading expert weights; quantising them
 // attacks that directly); jacopoparretti "Mixture of experts, token by token",
@@ -51,7 +53,9 @@ using tc::TcMaps;
 constexpr int CONV_WARPS = 8;
 constexpr int CONV_WARP0 = 6;
 constexpr int QPROD_WARP = CONV_WARP0 + CONV_WARPS;
-constexpr int NUM_THREADS = (QPROD_WARP + 1) * 32;
+constexpr int MMA2_WARP = QPROD_WARP + 1;  // issues matrix 1's MMAs (warp 1 issues matrix 0's)
+constexpr int NUM_THREADS = (MMA2_WARP + 1) * 32;
+constexpr int MMA_ISSUERS = 2;
 constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BAR_BYTES = 512;
@@ -72,7 +76,7 @@ struct WqShape {
   static constexpr int SMEM_BYTES = 1024 + NQ * Q_BYTES + NBS * B_BYTES + BAR_BYTES;
   static_assert(NA >= 2 && NQ >= 2, "rings");
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-  static_assert(2 * NQ + 2 * NBS + 2 * NA + 5 <= BAR_BYTES / 8 - 2, "barrier area");
+  static_assert(2 * NQ + 2 * NBS + 2 * NA + 6 <= BAR_BYTES / 8 - 2, "barrier area");
 };
 
 struct WqGroup {
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* q_base = smem;                               // NQ code stages
   uint8_t* b_base = q_base + NQ * Q_BYTES;              // NBS token boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(b_base + NBS * Sh::B_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NQ + 2 * NBS + 2 * NA + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NQ + 2 * NBS + 2 * NA + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int T0 = 2 * NQ + 2 * NBS + 2 * NA;
   auto tfull = [&](int a) { return bar0 + 8u * (T0 + a); };
   auto tempty = [&](int a) { return bar0 + 8u * (T0 + 2 + a); };
-  const uint32_t done_bar = bar0 + 8u * (T0 + 4);
+  const uint32_t done_bar = bar0 + 8u * (T0 + 4);  // one per MMA issuer
 
   const WqGroup& G = p.grp;
   if (threadIdx.x == 0) {
@@ -196,17 +200,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < NBS; ++i) {
       tc::mbar_init(bfull(i), 1);
-      tc::mbar_init(bempty(i), 1);
+      tc::mbar_init(bempty(i), MMA_ISSUERS);
     }
     for (int i = 0; i < NA; ++i) {
       tc::mbar_init(afull(i), CONV_WARPS);
-      tc::mbar_init(aempty(i), 1);
+      tc::mbar_init(aempty(i), MMA_ISSUERS);
     }
     for (int a = 0; a < 2; ++a) {
-      tc::mbar_init(tfull(a), 1);
+      tc::mbar_init(tfull(a), MMA_ISSUERS);
       tc::mbar_init(tempty(a), EPI_WARPS);
     }
-    tc::mbar_init(done_bar, 1);
+    for (int i = 0; i < MMA_ISSUERS; ++i) tc::mbar_init(done_bar + 8u * i, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -289,9 +293,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < NQ; ++i)
           if ((issued >> i) & 1u) tc::wait_drain(qfull(i), (par >> i) & 1u, abort_flag, drain_tmo);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == MMA2_WARP) {
+    // --------------------------------------------------------------- MMA issuers
+    // Two threads issue the tile's MMAs, one per weight matrix (its own D), so
+    // that the small MMAs of the swapped shape are issued twice as fast; both
+    // commit to the shared barriers (counts of two).
     if (lane == 0) {
+      const int mi = warp == 1 ? 0 : 1;
       constexpr uint32_t IDESC = tcf8::make_idesc_f16(BM, NB);
       int as = 0, bs = 0;
       uint32_t aph = 0, bph = 0, acc = 0, acc_phase = 0;
@@ -304,21 +312,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!tc::wait_bounded(tempty(acc), acc_phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc::tc_fence_after();
         for (int g = 0; g < nck; ++g) {
-          if (!tc::wait_bounded(afull(as), aph, abort_flag, tmo) ||
-              !tc::wait_bounded(bfull(bs), bph, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
+          // afull also covers the token box: the first converter warp waited for it
+          if (!tc::wait_fast(afull(as), aph, abort_flag, tmo)) { ok = false; break; }
           tc::tc_fence_after();
           const uint64_t bd = tc::sw128_kmajor_desc(b_0 + bs * Sh::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint32_t accum = (g | kk) != 0 ? 1u : 0u;
             // +32 bytes per K step in the B descriptor; +8 TMEM columns in A
-            tc_mma_ts(tmem_base + d_col(acc, 0), tmem_base + a_col(as, 0) + 8u * kk, bd + 2u * kk,
-                      IDESC, accum);
-            tc_mma_ts(tmem_base + d_col(acc, 1), tmem_base + a_col(as, 1) + 8u * kk, bd + 2u * kk,
-                      IDESC, accum);
+            tc_mma_ts(tmem_base + d_col(acc, mi), tmem_base + a_col(as, mi) + 8u * kk, bd + 2u * kk,
+                      IDESC, (g | kk) != 0 ? 1u : 0u);
           }
           tc::tc_commit(aempty(as));  // the decoded chunk has been read
           tc::tc_commit(bempty(bs));  // and the token box
@@ -330,8 +332,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc ^= 1u;
         if (acc == 0u) acc_phase ^= 1u;
       }
-      tc::tc_commit(done_bar);
-      tc::wait_drain(done_bar, 0u, abort_flag, drain_tmo);
+      tc::tc_commit(done_bar + 8u * mi);
+      tc::wait_drain(done_bar + 8u * mi, 0u, abort_flag, drain_tmo);
     }
   } else if (warp >= CONV_WARP0 && warp < CONV_WARP0 + CONV_WARPS) {
     // ---------------------------------------------------------------- converters
@@ -349,8 +351,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t q_row_off = qrow * Q_ROW;
     const int rsw = qrow & 7;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int qs = 0, as = 0;
-    uint32_t qph = 0, aph = 0;
+    int qs = 0, as = 0, bs_cv = 0;  // bs_cv: the token-box ring, followed by the first warp
+    uint32_t qph = 0, aph = 0, bph_cv = 0;
     bool ok = true;
     // MXFP4: this row's block exponents (this code stage's eight and the next
     // stage's, loaded one stage ahead) and 1 / its row factor
@@ -369,67 +371,98 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         inv_rf = valid ? 1.0f / __ldg(rf + (int64_t)ti.e * G.scale_stride + grow) : 0.f;
         bs_nxt = bsrow != nullptr ? __ldg(reinterpret_cast<const uint2*>(bsrow)) : make_uint2(0u, 0u);
       }
-      for (int g = 0; g < nck; ++g) {
-        const int h = g % QCH;
+      // two chunks per batch: one wait for both TMEM slots, two stores, one
+      // wait for the stores, both slots published together (the fixed
+      // latency of a batch is paid once per two chunks)
+      for (int g = 0; g < nck; g += 2) {
+        const int npair = nck - g < 2 ? nck - g : 2;
+        const int as1 = as + 1 == NA ? 0 : as + 1;
+        const uint32_t aph1 = as + 1 == NA ? aph ^ 1u : aph;
         int w = 1;
-        if (h == 0) {
-          // lane 0 waits for the code stage; the others then observe the completed
-          // phase themselves (it cannot move on before this warp releases it)
-          if (lane == 0) w = tc::wait_bounded(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
-          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-          (void)tc::mbar_try_wait(qfull(qs), qph);
-          if constexpr (WQ == tcf8::WQ_MXFP4) {
-            bs_cur = bs_nxt;
-            const int qn = g / QCH + 1;
-            if (qn < nqs && bsrow != nullptr)
-              bs_nxt = __ldg(reinterpret_cast<const uint2*>(bsrow + (size_t)qn * 8));
-          }
-        }
-        const uint8_t* qr = q_base + qs * Q_BYTES + q_row_off;
-        uint32_t o[32];
-        if constexpr (WQ == tcf8::WQ_MXFP4) {
-          uint2 c[4];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qr + (((2 * h + j) ^ rsw) << 4));
-            c[2 * j] = make_uint2(v.x, v.y);
-            c[2 * j + 1] = make_uint2(v.z, v.w);
-          }
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {  // blocks 2h + j of this code stage
-            const int blk = 2 * h + j;
-            const uint32_t wbs = blk < 4 ? bs_cur.x : bs_cur.y;
-            const uint32_t mult = tcf8::mx_block_multiplier((wbs >> (8 * (blk & 3))) & 0xFFu, inv_rf);
-            tcf8::mxfp4x16_to_f16x16(c[2 * j], mult, o + 16 * j);
-            tcf8::mxfp4x16_to_f16x16(c[2 * j + 1], mult, o + 16 * j + 8);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qr + (((4 * h + j) ^ rsw) << 4));
-            tcf8::e4m3x4_to_f16x4(v.x, o[8 * j], o[8 * j + 1]);
-            tcf8::e4m3x4_to_f16x4(v.y, o[8 * j + 2], o[8 * j + 3]);
-            tcf8::e4m3x4_to_f16x4(v.z, o[8 * j + 4], o[8 * j + 5]);
-            tcf8::e4m3x4_to_f16x4(v.w, o[8 * j + 6], o[8 * j + 7]);
-          }
-        }
-        if (h == QCH - 1 || g == nck - 1) {  // this code stage is fully read: hand it back
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(qempty(qs));
-          if (++qs == NQ) { qs = 0; qph ^= 1u; }
-        }
-        // wait for the chunk's TMEM slot, store the decoded row, publish it
-        if (lane == 0) w = tc::wait_bounded(aempty(as), aph ^ 1u, abort_flag, tmo) ? 1 : 0;
+        if (lane == 0)
+          w = (tc::wait_fast(aempty(as), aph ^ 1u, abort_flag, tmo) &&
+               (npair < 2 || tc::wait_fast(aempty(as1), aph1 ^ 1u, abort_flag, tmo)))
+                  ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
         tc::tc_fence_after();
-        tmem_st32(tmem_base + lane_base + a_col(as, m), o);
+        uint32_t o[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c >= npair) break;
+          const int h = (g + c) % QCH;
+          if (h == 0) {
+            // lane 0 waits for the code stage; the others then observe the completed
+            // phase themselves (it cannot move on before this warp releases it)
+            if (lane == 0) w = tc::wait_fast(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+            (void)tc::mbar_try_wait(qfull(qs), qph);
+            if constexpr (WQ == tcf8::WQ_MXFP4) {
+              bs_cur = bs_nxt;
+              const int qn = (g + c) / QCH + 1;
+              if (qn < nqs && bsrow != nullptr)
+                bs_nxt = __ldg(reinterpret_cast<const uint2*>(bsrow + (size_t)qn * 8));
+            }
+          }
+          const uint8_t* qr = q_base + qs * Q_BYTES + q_row_off;
+          if constexpr (WQ == tcf8::WQ_MXFP4) {
+            uint2 cc[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint4 v = *reinterpret_cast<const uint4*>(qr + (((2 * h + j) ^ rsw) << 4));
+              cc[2 * j] = make_uint2(v.x, v.y);
+              cc[2 * j + 1] = make_uint2(v.z, v.w);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // blocks 2h + j of this code stage
+              const int blk = 2 * h + j;
+              const uint32_t wbs = blk < 4 ? bs_cur.x : bs_cur.y;
+              const uint32_t mult =
+                  tcf8::mx_block_multiplier((wbs >> (8 * (blk & 3))) & 0xFFu, inv_rf);
+              tcf8::mxfp4x16_to_f16x16(cc[2 * j], mult, o[c] + 16 * j);
+              tcf8::mxfp4x16_to_f16x16(cc[2 * j + 1], mult, o[c] + 16 * j + 8);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 v = *reinterpret_cast<const uint4*>(qr + (((4 * h + j) ^ rsw) << 4));
+              tcf8::e4m3x4_to_f16x4(v.x, o[c][8 * j], o[c][8 * j + 1]);
+              tcf8::e4m3x4_to_f16x4(v.y, o[c][8 * j + 2], o[c][8 * j + 3]);
+              tcf8::e4m3x4_to_f16x4(v.z, o[c][8 * j + 4], o[c][8 * j + 5]);
+              tcf8::e4m3x4_to_f16x4(v.w, o[c][8 * j + 6], o[c][8 * j + 7]);
+            }
+          }
+          if (h == QCH - 1 || g + c == nck - 1) {  // this code stage is fully read
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(qempty(qs));
+            if (++qs == NQ) { qs = 0; qph ^= 1u; }
+          }
+          tmem_st32(tmem_base + lane_base + a_col(c == 0 ? as : as1, m), o[c]);
+        }
+        if (!ok) break;
+        // the first converter warp also vouches for the batch's token boxes, so
+        // the MMA thread waits on one barrier per chunk
+        if (warp == CONV_WARP0 && lane == 0) {
+          for (int c = 0; c < npair && ok; ++c) {
+            const int bsc = (bs_cv + c) % NBS;
+            const uint32_t bphc = ((bs_cv + c) / NBS) & 1u ? bph_cv ^ 1u : bph_cv;
+            if (!tc::wait_fast(bfull(bsc), bphc, abort_flag, tmo)) ok = false;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
         tmem_st_wait();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(afull(as));
-        if (++as == NA) { as = 0; aph ^= 1u; }
+        if (lane == 0) {
+          tc::mbar_arrive(afull(as));
+          if (npair == 2) tc::mbar_arrive(afull(as1));
+        }
+        for (int c = 0; c < npair; ++c) {
+          if (++as == NA) { as = 0; aph ^= 1u; }
+          if (++bs_cv == NBS) { bs_cv = 0; bph_cv ^= 1u; }
+        }
       }
     }
+    tmem_st_wait();  // an aborted batch may have stores in flight: TMEM is freed below
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
