@@ -30,10 +30,14 @@
 // issuer of matrix 1.
 // Synchronisation, all waits bounded:
 //   qfull[q]  code producer expect_tx + TMA bytes;     qempty[q] 8 converter warps
-//   bfull[b]  activation producer expect_tx + bytes (waited by the first
-//             converter warp);                          bempty[b] 2 MMA commits
+//   bfull[b]  activation producer expect_tx + bytes;   bempty[b] 2 MMA commits
 //   afull[a]  8 converter warps (after tcgen05.st, wait::st and the tcgen05
 //             fence);                                   aempty[a] 2 MMA commits
+// The ring of decoded chunks in TMEM is short (six slots at N = 32), so its
+// round trip (decode, store, publish, MMA issue, MMA completion, release) sets
+// the pace: every chunk is published on its own as soon as it is stored, and
+// the token box is checked by the MMA threads, not by a converter warp (the
+// slowest of the eight converter warps gates every chunk).
 //   tfull[2]  2 MMA commits;                            tempty[2] 4 epilogue warps
 // Sources: AI Engineering Illustrated "Mixture of Experts", "Trade-offs to
 // weigh" (small-batch MoE is bound by reading expert weights; quantising them
@@ -312,8 +316,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!tc::wait_bounded(tempty(acc), acc_phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         tc::tc_fence_after();
         for (int g = 0; g < nck; ++g) {
-          // afull also covers the token box: the first converter warp waited for it
           if (!tc::wait_fast(afull(as), aph, abort_flag, tmo)) { ok = false; break; }
+          if (!tc::wait_fast(bfull(bs), bph, abort_flag, tmo)) { ok = false; break; }
           tc::tc_fence_after();
           const uint64_t bd = tc::sw128_kmajor_desc(b_0 + bs * Sh::B_BYTES);
 #pragma unroll
@@ -351,8 +355,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t q_row_off = qrow * Q_ROW;
     const int rsw = qrow & 7;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int qs = 0, as = 0, bs_cv = 0;  // bs_cv: the token-box ring, followed by the first warp
-    uint32_t qph = 0, aph = 0, bph_cv = 0;
+    int qs = 0, as = 0;
+    uint32_t qph = 0, aph = 0;
     bool ok = true;
     // MXFP4: this row's block exponents (this code stage's eight and the next
     // stage's, loaded one stage ahead) and 1 / its row factor
@@ -371,98 +375,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         inv_rf = valid ? 1.0f / __ldg(rf + (int64_t)ti.e * G.scale_stride + grow) : 0.f;
         bs_nxt = bsrow != nullptr ? __ldg(reinterpret_cast<const uint2*>(bsrow)) : make_uint2(0u, 0u);
       }
-      // two chunks per batch: one wait for both TMEM slots, two stores, one
-      // wait for the stores, both slots published together (the fixed
-      // latency of a batch is paid once per two chunks)
-      for (int g = 0; g < nck; g += 2) {
-        const int npair = nck - g < 2 ? nck - g : 2;
-        const int as1 = as + 1 == NA ? 0 : as + 1;
-        const uint32_t aph1 = as + 1 == NA ? aph ^ 1u : aph;
+      for (int g = 0; g < nck; ++g) {
+        const int h = g % QCH;
         int w = 1;
-        if (lane == 0)
-          w = (tc::wait_fast(aempty(as), aph ^ 1u, abort_flag, tmo) &&
-               (npair < 2 || tc::wait_fast(aempty(as1), aph1 ^ 1u, abort_flag, tmo)))
-                  ? 1 : 0;
+        if (lane == 0) w = tc::wait_fast(aempty(as), aph ^ 1u, abort_flag, tmo) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
         tc::tc_fence_after();
-        uint32_t o[2][32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (c >= npair) break;
-          const int h = (g + c) % QCH;
-          if (h == 0) {
-            // lane 0 waits for the code stage; the others then observe the completed
-            // phase themselves (it cannot move on before this warp releases it)
-            if (lane == 0) w = tc::wait_fast(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-            (void)tc::mbar_try_wait(qfull(qs), qph);
-            if constexpr (WQ == tcf8::WQ_MXFP4) {
-              bs_cur = bs_nxt;
-              const int qn = (g + c) / QCH + 1;
-              if (qn < nqs && bsrow != nullptr)
-                bs_nxt = __ldg(reinterpret_cast<const uint2*>(bsrow + (size_t)qn * 8));
-            }
-          }
-          const uint8_t* qr = q_base + qs * Q_BYTES + q_row_off;
+        if (h == 0) {
+          // lane 0 waits for the code stage; the others then observe the completed
+          // phase themselves (it cannot move on before this warp releases it)
+          if (lane == 0) w = tc::wait_fast(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+          (void)tc::mbar_try_wait(qfull(qs), qph);
           if constexpr (WQ == tcf8::WQ_MXFP4) {
-            uint2 cc[4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const uint4 v = *reinterpret_cast<const uint4*>(qr + (((2 * h + j) ^ rsw) << 4));
-              cc[2 * j] = make_uint2(v.x, v.y);
-              cc[2 * j + 1] = make_uint2(v.z, v.w);
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {  // blocks 2h + j of this code stage
-              const int blk = 2 * h + j;
-              const uint32_t wbs = blk < 4 ? bs_cur.x : bs_cur.y;
-              const uint32_t mult =
-                  tcf8::mx_block_multiplier((wbs >> (8 * (blk & 3))) & 0xFFu, inv_rf);
-              tcf8::mxfp4x16_to_f16x16(cc[2 * j], mult, o[c] + 16 * j);
-              tcf8::mxfp4x16_to_f16x16(cc[2 * j + 1], mult, o[c] + 16 * j + 8);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 v = *reinterpret_cast<const uint4*>(qr + (((4 * h + j) ^ rsw) << 4));
-              tcf8::e4m3x4_to_f16x4(v.x, o[c][8 * j], o[c][8 * j + 1]);
-              tcf8::e4m3x4_to_f16x4(v.y, o[c][8 * j + 2], o[c][8 * j + 3]);
-              tcf8::e4m3x4_to_f16x4(v.z, o[c][8 * j + 4], o[c][8 * j + 5]);
-              tcf8::e4m3x4_to_f16x4(v.w, o[c][8 * j + 6], o[c][8 * j + 7]);
-            }
-          }
-          if (h == QCH - 1 || g + c == nck - 1) {  // this code stage is fully read
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(qempty(qs));
-            if (++qs == NQ) { qs = 0; qph ^= 1u; }
-          }
-          tmem_st32(tmem_base + lane_base + a_col(c == 0 ? as : as1, m), o[c]);
-        }
-        if (!ok) break;
-        // the first converter warp also vouches for the batch's token boxes, so
-        // the MMA thread waits on one barrier per chunk
-        if (warp == CONV_WARP0 && lane == 0) {
-          for (int c = 0; c < npair && ok; ++c) {
-            const int bsc = (bs_cv + c) % NBS;
-            const uint32_t bphc = ((bs_cv + c) / NBS) & 1u ? bph_cv ^ 1u : bph_cv;
-            if (!tc::wait_fast(bfull(bsc), bphc, abort_flag, tmo)) ok = false;
+            bs_cur = bs_nxt;
+            const int qn = g / QCH + 1;
+            if (qn < nqs && bsrow != nullptr)
+              bs_nxt = __ldg(reinterpret_cast<const uint2*>(bsrow + (size_t)qn * 8));
           }
         }
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
+        uint32_t o[32];
+        const uint8_t* qr = q_base + qs * Q_BYTES + q_row_off;
+        if constexpr (WQ == tcf8::WQ_MXFP4) {
+          uint2 cc[4];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qr + (((2 * h + j) ^ rsw) << 4));
+            cc[2 * j] = make_uint2(v.x, v.y);
+            cc[2 * j + 1] = make_uint2(v.z, v.w);
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {  // blocks 2h + j of this code stage
+            const int blk = 2 * h + j;
+            const uint32_t wbs = blk < 4 ? bs_cur.x : bs_cur.y;
+            const uint32_t mult =
+                tcf8::mx_block_multiplier((wbs >> (8 * (blk & 3))) & 0xFFu, inv_rf);
+            tcf8::mxfp4x16_to_f16x16(cc[2 * j], mult, o + 16 * j);
+            tcf8::mxfp4x16_to_f16x16(cc[2 * j + 1], mult, o + 16 * j + 8);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qr + (((4 * h + j) ^ rsw) << 4));
+            tcf8::e4m3x4_to_f16x4(v.x, o[8 * j], o[8 * j + 1]);
+            tcf8::e4m3x4_to_f16x4(v.y, o[8 * j + 2], o[8 * j + 3]);
+            tcf8::e4m3x4_to_f16x4(v.z, o[8 * j + 4], o[8 * j + 5]);
+            tcf8::e4m3x4_to_f16x4(v.w, o[8 * j + 6], o[8 * j + 7]);
+          }
+        }
+        if (h == QCH - 1 || g == nck - 1) {  // this code stage is fully read
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(qempty(qs));
+          if (++qs == NQ) { qs = 0; qph ^= 1u; }
+        }
+        tmem_st32(tmem_base + lane_base + a_col(as, m), o);
         tmem_st_wait();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          tc::mbar_arrive(afull(as));
-          if (npair == 2) tc::mbar_arrive(afull(as1));
-        }
-        for (int c = 0; c < npair; ++c) {
-          if (++as == NA) { as = 0; aph ^= 1u; }
-          if (++bs_cv == NBS) { bs_cv = 0; bph_cv ^= 1u; }
-        }
+        if (lane == 0) tc::mbar_arrive(afull(as));
+        if (++as == NA) { as = 0; aph ^= 1u; }
       }
     }
-    tmem_st_wait();  // an aborted batch may have stores in flight: TMEM is freed below
+    tmem_st_wait();  // an aborted chunk may have stores in flight: TMEM is freed below
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
