@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         const int stage = kb % STAGES;
         const uint32_t phase = (uint32_t)((kb / STAGES) & 1);
-        if (!tc::wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+        if (!tc::wait_fast(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
         const uint32_t sa = stage0 + stage * STAGE_BYTES;
         const uint32_t fb = full_bar(stage);
         tc::mbar_expect_tx(fb, A_BYTES + 3 * b_bytes);
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kend = min(nkb, (ch + 1) * KC);
         for (int first = 1; kb < kend; ++kb, first = 0) {
           const int stage = kb % STAGES;
-          if (!tc::wait_bounded(full_bar(stage), (uint32_t)((kb / STAGES) & 1), abort_flag, tmo)) {
+          if (!tc::wait_fast(full_bar(stage), (uint32_t)((kb / STAGES) & 1), abort_flag, tmo)) {
             ok = false;
             break;
           }

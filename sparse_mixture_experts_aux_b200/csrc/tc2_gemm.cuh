@@ -171,6 +171,14 @@ __device__ __noinline__ bool wait_pair(uint32_t bar, uint32_t parity, volatile i
   }
 }
 
+// The same with the first test inline: a phase that has already completed
+// costs one try_wait instead of a call (the issuing threads of the main loop
+// wait once per K step).
+__device__ __forceinline__ bool wait_pair_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               uint32_t peer_abort, unsigned long long timeout_ns) {
+  return tc::mbar_try_wait(bar, parity) || wait_pair(bar, parity, abort_flag, peer_abort, timeout_ns);
+}
+
 struct PairTile {
   int g, e, row0, nb;
   bool half_valid[2];
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kbs = p.g[ti.g].k_blocks;
         const int arow = ti.row0 + HALF_M * (int)rank;
         for (int kb = 0; kb < kbs; ++kb) {
-          if (!wait_pair(empty_bar(stage), phase ^ 1u, abort_flag, peer_abort, tmo)) {
+          if (!wait_pair_fast(empty_bar(stage), phase ^ 1u, abort_flag, peer_abort, tmo)) {
             ok = false;
             break;
           }
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kbs; ++kb) {
-          if (!wait_pair(full_bar(stage), phase, abort_flag, peer_abort, tmo)) {
+          if (!wait_pair_fast(full_bar(stage), phase, abort_flag, peer_abort, tmo)) {
             ok = false;
             break;
           }

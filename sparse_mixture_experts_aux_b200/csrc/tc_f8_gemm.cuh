@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         for (int st = 0; st < nst; ++st) {
-          if (!tc::wait_bounded(aempty(as), aph ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!tc::wait_fast(aempty(as), aph ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const int nv = min(CH, nck - st * CH);
           tc::mbar_expect_tx(afull(as), nv * Sh::A_SUB);
           for (int c = 0; c < nv; ++c)
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const tc::TileInfo ti = decode_tile_f8(tile, G, s_ts);
         if (tc::tile_out_of_bounds(ti.e, ti.nb, ti.row0, BM, G)) continue;
         for (int qi = 0; qi < nqs; ++qi) {
-          if (!tc::wait_bounded(qempty(qs), qph ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!tc::wait_fast(qempty(qs), qph ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const uint32_t dq = q_0 + qs * Sh::Q_BYTES;
           const int x = qi * (Sh::Q_ROW / 4);  // the codes are described as 32-bit words
           tc::mbar_expect_tx(qfull(qs), Sh::Q_BYTES);
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int st = 0; st < nst; ++st) {
-          if (!tc::wait_bounded(full(ss), sph, abort_flag, tmo)) { ok = false; break; }
+          if (!tc::wait_fast(full(ss), sph, abort_flag, tmo)) { ok = false; break; }
           tc::tc_fence_after();
           const int nv = min(CH, nck - st * CH);
           for (int c = 0; c < nv; ++c) {
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // lane 0 waits (bounded) for the stage's slot to be free; __syncwarp
         // then orders the other lanes' writes after it
         int w = 1;
-        if (lane == 0) w = tc::wait_bounded(empty(ss), sph ^ 1u, abort_flag, tmo) ? 1 : 0;
+        if (lane == 0) w = tc::wait_fast(empty(ss), sph ^ 1u, abort_flag, tmo) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
         const int nv = min(CH, nck - st * CH);
         uint8_t* const bst = s_base + ss * Sh::S_BYTES + b_row;
@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // phase themselves (it cannot move on before this warp releases it),
             // which gives each lane its own acquire for the TMA-written bytes
             w = 1;
-            if (lane == 0) w = tc::wait_bounded(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
+            if (lane == 0) w = tc::wait_fast(qfull(qs), qph, abort_flag, tmo) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
             (void)tc::mbar_try_wait(qfull(qs), qph);
             if constexpr (WQ == WQ_MXFP4) {

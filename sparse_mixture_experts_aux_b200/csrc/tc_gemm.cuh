@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if ((uint32_t)(gs & 1) != me) continue;
           const int stage = (int)(gs % STAGES);
           const uint32_t phase = (uint32_t)((gs / STAGES) & 1);
-          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
+          if (!wait_fast(empty_bar(stage), phase ^ 1u, abort_flag, tmo)) { ok = false; break; }
           const uint32_t sa = stage0 + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full_bar(stage);
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kbs; ++kb) {
-          if (!wait_bounded(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
+          if (!wait_fast(full_bar(stage), phase, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = stage0 + stage * STAGE_BYTES;
           const uint64_t ad = sw128_kmajor_desc(sa);
