@@ -14,7 +14,7 @@
 #include "permute.cuh"
 #include "tc_gemm.cuh"
 #include "tc2_gemm.cuh"
-#include "tc_f8_gemm.cuh"
+#include "quant_formats.cuh"
 #include "router_tc.cuh"
 #include "tc_wq_swap.cuh"
 
@@ -215,38 +215,8 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int EPI, int AR, int WQ>
-bool f8_attr() {
-  return cudaFuncSetAttribute(moe::tcf8::tc_f8_grouped_gemm_kernel<EPI, AR, WQ>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              moe::tcf8::F8Shape<AR, WQ>::SMEM_BYTES) == cudaSuccess;
-}
-
-template <int WQ>
-bool f8_attrs() {
-  using moe::tc::EPI_SWIGLU_TC;
-  using moe::tc::EPI_SCALE_TC;
-  return f8_attr<EPI_SWIGLU_TC, 128, WQ>() && f8_attr<EPI_SCALE_TC, 128, WQ>() &&
-         f8_attr<EPI_SWIGLU_TC, 64, WQ>() && f8_attr<EPI_SCALE_TC, 64, WQ>() &&
-         f8_attr<EPI_SWIGLU_TC, 32, WQ>() && f8_attr<EPI_SCALE_TC, 32, WQ>();
-}
-
-// Quantised-weight grouped GEMM (WQ: FP8 or MXFP4 codes) with an activation box
-// of `ar` rows.
-template <int EPI, int WQ>
-void launch_f8(int ar, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
-               const moe::tcf8::F8Params& fp) {
-  using namespace moe::tcf8;
-  if (ar == 32)
-    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 32, WQ>, grid, NUM_THREADS, F8Shape<32, WQ>::SMEM_BYTES, st, maps, fp);
-  else if (ar == 64)
-    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 64, WQ>, grid, NUM_THREADS, F8Shape<64, WQ>::SMEM_BYTES, st, maps, fp);
-  else
-    launch_pdl(tc_f8_grouped_gemm_kernel<EPI, 128, WQ>, grid, NUM_THREADS, F8Shape<128, WQ>::SMEM_BYTES, st, maps, fp);
-}
-
-// Quantised-weight grouped GEMM for at most 64 tokens (operands swapped,
-// decoded weights in TMEM) with token boxes of `nb` rows (32 or 64).
+// Quantised-weight grouped GEMM (operands swapped, decoded weights in TMEM)
+// with token boxes of `nb` rows (32, 64 or 128).
 template <int EPI, int WQ>
 bool wq_attr() {
   return cudaFuncSetAttribute(moe::wqs::tc_wq_swap_kernel<EPI, 32, WQ>,
@@ -254,7 +224,10 @@ bool wq_attr() {
                               moe::wqs::WqShape<32, WQ>::SMEM_BYTES) == cudaSuccess &&
          cudaFuncSetAttribute(moe::wqs::tc_wq_swap_kernel<EPI, 64, WQ>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              moe::wqs::WqShape<64, WQ>::SMEM_BYTES) == cudaSuccess;
+                              moe::wqs::WqShape<64, WQ>::SMEM_BYTES) == cudaSuccess &&
+         cudaFuncSetAttribute(moe::wqs::tc_wq_swap_kernel<EPI, 128, WQ>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moe::wqs::WqShape<128, WQ>::SMEM_BYTES) == cudaSuccess;
 }
 
 template <int EPI, int WQ>
@@ -264,9 +237,12 @@ void launch_wq(int nb, int grid, cudaStream_t st, const moe::tc::TcMaps& maps,
   if (nb == 32)
     launch_pdl(tc_wq_swap_kernel<EPI, 32, WQ>, grid, NUM_THREADS, WqShape<32, WQ>::SMEM_BYTES, st,
                maps, wp);
-  else
+  else if (nb == 64)
     launch_pdl(tc_wq_swap_kernel<EPI, 64, WQ>, grid, NUM_THREADS, WqShape<64, WQ>::SMEM_BYTES, st,
                maps, wp);
+  else
+    launch_pdl(tc_wq_swap_kernel<EPI, 128, WQ>, grid, NUM_THREADS, WqShape<128, WQ>::SMEM_BYTES,
+               st, maps, wp);
 }
 
 // 1-CTA grouped GEMM with an activation box of `ar` rows (128, 64 or 32);
@@ -344,7 +320,6 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 64, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 64, true>() ||
         !tc_attr<moe::tc::EPI_SWIGLU_TC, 32, true>() || !tc_attr<moe::tc::EPI_SCALE_TC, 32, true>())
       return MOE_ERR_CUDA;
-    if (!f8_attrs<moe::tcf8::WQ_FP8>() || !f8_attrs<moe::tcf8::WQ_MXFP4>()) return MOE_ERR_CUDA;
     if (!wq_attr<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_FP8>() ||
         !wq_attr<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>() ||
         !wq_attr<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>() ||
@@ -419,7 +394,7 @@ bool encode_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mi
                    uint32_t box_rows) {
   cuuint64_t dims[3] = {inner / 4, mid, outer};
   cuuint64_t strides[2] = {inner, inner * mid};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::tcf8::F8Shape<128>::Q_ROW / 4), box_rows, 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::wqs::Q_ROW / 4), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r =
       g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box,
@@ -685,11 +660,11 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       tm.at(11);
       if (launched() != MOE_OK) return MOE_ERR_CUDA;
     } else if (dims->weight_format == MOE_WEIGHTS_FP8 || dims->weight_format == MOE_WEIGHTS_MXFP4) {
-      // FP8 or MXFP4 expert weights: 1-CTA kernels that dequantise the weight
-      // tiles on chip; at most 64 tokens: operands swapped, decoded weights in TMEM
+      // FP8 or MXFP4 expert weights: operands swapped (weights are the M = 128
+      // side), decoded on chip into TMEM; token boxes of 32, 64 or 128 rows
       const bool mx = dims->weight_format == MOE_WEIGHTS_MXFP4;
-      if (P.T <= 64) {
-        const int nb = P.T <= 32 ? 32 : 64;
+      {
+        const int nb = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
         const float* sc = dims->weight_scales;
         const size_t gsz = static_cast<size_t>(E) * P.de;
         const int cpb = mx ? 2 : 1;  // codes per byte
@@ -748,69 +723,7 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
           launch_wq<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>(nb, num_sms, st, dn, wd);
         tm.at(11);
         if (launched() != MOE_OK) return MOE_ERR_CUDA;
-      } else {
-      const int arows = P.T <= 32 ? 32 : (P.T <= 64 ? 64 : 128);
-      const float* sc = dims->weight_scales;
-      const size_t gsz = static_cast<size_t>(E) * P.de;
-      const int cpb = mx ? 2 : 1;  // codes per byte
-      moe::tc::TcMaps up, dn;
-      memset(&up, 0, sizeof(up));
-      memset(&dn, 0, sizeof(dn));
-      const bool ok = encode_map(&up.a[0], xp, P.d, P.rows_max, 1, arows, 2) &&
-                      encode_map_u8(&up.b0[0], W_g, P.d / cpb, P.de, E, moe::tc::BN / 2) &&
-                      encode_map_u8(&up.b1[0], W_u, P.d / cpb, P.de, E, moe::tc::BN / 2) &&
-                      encode_map(&dn.a[0], h, P.de, P.rows_max, 1, arows, 2) &&
-                      encode_map_u8(&dn.b0[0], W_d, P.de / cpb, P.d, E, moe::tc::BN);
-      if (!ok) return MOE_ERR_CUDA;
-      dn.b1[0] = dn.b0[0];
-      // MXFP4 block exponents: [W_g | W_u | W_d], K / 32 bytes per weight row
-      const uint8_t* bs = dims->weight_block_scales;
-      const size_t gbs = gsz * (P.d / 32);
-      moe::tcf8::F8Params fu{};
-      fu.timeout_ns = wait_tmo;
-      fu.drain_timeout_ns = kDrainTimeoutNs;
-      fu.call_err = call_err;
-      fu.grp.g = {tile_start, E, rows_cap, (P.de + moe::tc::BN / 2 - 1) / (moe::tc::BN / 2),
-                  P.d / moe::tc::BK, P.de, h, nullptr};
-      fu.grp.scale0 = sc;
-      fu.grp.scale1 = sc + gsz;
-      fu.grp.scale_stride = P.de;
-      if (mx) {
-        fu.grp.bscale0 = bs;
-        fu.grp.bscale1 = bs + gbs;
-        fu.grp.bscale_stride = static_cast<int64_t>(P.de) * (P.d / 32);
-        fu.grp.kblk = P.d / 32;
       }
-      moe::tcf8::F8Params fd{};
-      fd.timeout_ns = wait_tmo;
-      fd.drain_timeout_ns = kDrainTimeoutNs;
-      fd.call_err = call_err;
-      fd.grp.g = {tile_start, E, rows_cap, (P.d + moe::tc::BN - 1) / moe::tc::BN,
-                  P.de / moe::tc::BK, P.d, yrows, rowgate};
-      fd.grp.scale0 = sc + 2 * gsz;
-      fd.grp.scale1 = sc + 2 * gsz;
-      fd.grp.scale_stride = P.d;
-      if (mx) {
-        fd.grp.bscale0 = bs + 2 * gbs;
-        fd.grp.bscale1 = bs + 2 * gbs;
-        fd.grp.bscale_stride = static_cast<int64_t>(P.d) * (P.de / 32);
-        fd.grp.kblk = P.de / 32;
-      }
-      tm.at(8);
-      if (mx)
-        launch_f8<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>(arows, num_sms, st, up, fu);
-      else
-        launch_f8<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_FP8>(arows, num_sms, st, up, fu);
-      tm.at(9);
-      if (launched() != MOE_OK) return MOE_ERR_CUDA;
-      tm.at(10);
-      if (mx)
-        launch_f8<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_MXFP4>(arows, num_sms, st, dn, fd);
-      else
-        launch_f8<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_FP8>(arows, num_sms, st, dn, fd);
-      tm.at(11);
-      if (launched() != MOE_OK) return MOE_ERR_CUDA;
-      }  // more than 64 tokens
     } else {
     // (4) gate/up projection + SwiGLU, (5) down projection scaled by the gates.
     // CTA-pair tiles (256 rows) cut the operand traffic per SM by a third but

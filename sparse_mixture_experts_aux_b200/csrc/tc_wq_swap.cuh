@@ -1,24 +1,29 @@
-// Grouped expert GEMMs with quantised expert weights (FP8 or MXFP4) for small
-// batches (at most 64 tokens): operands swapped, decoded weights in TMEM.
+// Grouped expert GEMMs with quantised expert weights (FP8 or MXFP4): operands
+// swapped, decoded weights in TMEM.
 //
-// At the weight-streaming (decode) shape every expert holds a handful of token
-// rows, so the weights are the large operand. Here they are the MMA's A operand
-// (M = 128 weight rows) and the token rows are B (N = 32 or 64, the activation
-// box), so one MMA step costs an eighth (a quarter) of the 128 x 256 step of
-// the general kernel. Each converter thread owns one weight row: it reads the
+// The weights are the MMA's A operand (M = 128 weight rows) and the token rows
+// are B (N = 32, 64 or 128, the activation box, chosen by the batch size). At
+// the weight-streaming (decode) shape every expert holds a handful of token
+// rows, and a 32-row box makes one MMA step an eighth of a 128 x 256 step; at
+// prefill a 128-row box gives each 64-deep chunk 512 tensor cycles against
+// about 300 cycles of decoding, and the token tile is the innermost index of
+// the tile walk, so concurrent tiles share a weight tile through L2. Each
+// converter thread owns one weight row: it reads the
 // row's codes from the shared-memory code ring, decodes them to fp16 in
 // registers (FP8: hardware e4m3x2 conversion; MXFP4: e2m1x2 conversion times
 // the block's 2^(X - X_row)), and stores them straight into TMEM with
 // tcgen05.st, where the MMA reads A (tcgen05.mma with A in tensor memory).
 // Decoded weights therefore never touch shared memory, which holds only codes
-// (six stages, 192 KB at N = 32) and activation boxes, and TMEM holds up to six
-// decoded 64-deep chunks ahead of the MMA.
+// (six stages, 192 KB at N = 32; four at N = 128) and activation boxes, and
+// TMEM holds up to six (N = 128: four) decoded 64-deep chunks ahead of the MMA.
 //
-// Tile: one expert's token rows (one activation box of N rows starting at its
-// segment) against two 128-row weight matrices: gate/up = W_g and W_u rows
-// [128 nb, 128 nb + 128), down = W_d rows [256 nb, 256 nb + 256) as two halves.
-// D holds, per matrix, 128 weight rows (TMEM lanes) x N tokens (columns),
-// double buffered, so one tile's epilogue overlaps the next tile's MMAs.
+// Tile: one 128-row tile of an expert's segment of routed rows, of which the
+// activation box loads the first N (at N = 32 or 64 the batch holds at most N
+// rows, so a segment is one tile and its rows fit the box), against two
+// 128-row weight matrices: gate/up = W_g and W_u rows [128 nb, 128 nb + 128),
+// down = W_d rows [256 nb, 256 nb + 256) as two halves. D holds, per matrix,
+// 128 weight rows (TMEM lanes) x N tokens (columns), double buffered at N <= 64
+// so one tile's epilogue overlaps the next tile's MMAs (single at N = 128).
 // Epilogue: lane j = weight row, column c = token: gate/up writes
 // H[c][j] = SiLU(g s_g) (u s_u) as fp16; down writes Yrows[c][j] =
 // gate_c (d s_d) as bf16, s_* the per-row weight scale (FP8) or row factor
@@ -44,7 +49,7 @@
 // attacks that directly); jacopoparretti "Mixture of experts, token by token",
 // "Memory".
 #pragma once
-#include "tc_f8_gemm.cuh"
+#include "quant_formats.cuh"
 
 namespace moe {
 namespace wqs {
@@ -67,14 +72,18 @@ constexpr int Q_ROW = 128;                  // bytes per weight row in a code st
 constexpr int Q_BYTES = 2 * BM * Q_ROW;     // two 128-row matrices: 32 KB
 constexpr int A_COLS = 2 * (BK / 2);        // TMEM columns of one decoded chunk (2 matrices)
 
-// Shape for token boxes of NB rows (32 or 64) and weight format WQ.
+// Shape for token boxes of NB rows (32, 64 or 128) and weight format WQ. With
+// 128-row boxes two accumulators would fill TMEM, so D is single-buffered there
+// (the epilogue then does not overlap the next tile's MMAs) and four decoded
+// chunks fit beside it.
 template <int NB, int WQ>
 struct WqShape {
-  static_assert(NB == 32 || NB == 64, "token box rows");
+  static_assert(NB == 32 || NB == 64 || NB == 128, "token box rows");
   static constexpr int QCH = WQ == tcf8::WQ_MXFP4 ? 4 : 2;  // 64-deep chunks per code stage
   static constexpr int B_BYTES = NB * BK * 2;               // fp16 token box of one chunk
-  static constexpr int NBS = 8;                             // token boxes in flight
-  static constexpr int D_COLS = 2 * 2 * NB;                 // 2 buffers x 2 matrices x NB
+  static constexpr int NBS = NB == 128 ? 6 : 8;             // token boxes in flight
+  static constexpr int NACC = NB == 128 ? 1 : 2;            // accumulator buffers
+  static constexpr int D_COLS = NACC * 2 * NB;              // buffers x 2 matrices x NB
   static constexpr int NA = (TMEM_COLS - D_COLS) / A_COLS;  // decoded chunks in TMEM
   static constexpr int NQ = (232448 - 1024 - BAR_BYTES - NBS * B_BYTES) / Q_BYTES;
   static constexpr int SMEM_BYTES = 1024 + NQ * Q_BYTES + NBS * B_BYTES + BAR_BYTES;
@@ -333,8 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         tc::tc_commit(tfull(acc));
-        acc ^= 1u;
-        if (acc == 0u) acc_phase ^= 1u;
+        if (++acc == (uint32_t)Sh::NACC) { acc = 0; acc_phase ^= 1u; }
       }
       tc::tc_commit(done_bar + 8u * mi);
       tc::wait_drain(done_bar + 8u * mi, 0u, abort_flag, drain_tmo);
@@ -490,8 +498,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty(acc));
-      acc ^= 1u;
-      if (acc == 0u) acc_phase ^= 1u;
+      if (++acc == (uint32_t)Sh::NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
