@@ -38,11 +38,25 @@ METRIC = "MoE-layer tokens/s and active TFLOP/s vs B200 bf16 roofline, Mixtral s
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# (workload, weights) -> DRAM bytes / algorithmic bytes of the gate/up kernel, from one ncu
-# capture of that kernel as built (profiles/); absent = not captured for the current build.
-TRAFFIC_RATIO = {("mixtral", "dtype"): 539.386880 / 545.259520}
-# the same for the down kernel (CTA pairs), T=1024 E=2 case: DRAM 344.265 MB / 310.4 MB
-DOWN_TRAFFIC_RATIO = {("mixtral", "dtype"): 344.265216 / 310.378496}
+# (workload, weights) -> (DRAM bytes / algorithmic bytes of the gate/up kernel, the case the
+# ratio was captured on), from one ncu capture of that kernel as built on a small case with
+# the same rows per expert and kernel choice; absent = not captured for the current build.
+# Algorithmic bytes are step_work's on the captured case (two experts).
+_PREFILL_CASE = "T=1024 E=2 case (1024 rows per expert)"
+_DECODE_CASE = "T=32 E=2 case"
+TRAFFIC_RATIO = {
+    ("mixtral", "dtype"): (538.84 / 545.26, _PREFILL_CASE),
+    ("mixtral", "fp8"): (300.30 / 310.60, _PREFILL_CASE),
+    ("decode", "fp8"): (240.30 / 237.46, _DECODE_CASE),
+    ("decode", "mxfp4"): (131.30 / 127.43, _DECODE_CASE),
+}
+# the same for the down kernel
+DOWN_TRAFFIC_RATIO = {
+    ("mixtral", "dtype"): (344.20 / 310.38, _PREFILL_CASE),
+    ("mixtral", "fp8"): (220.10 / 192.97, _PREFILL_CASE),
+    ("decode", "fp8"): (124.10 / 119.83, _DECODE_CASE),
+    ("decode", "mxfp4"): (65.90 / 64.79, _DECODE_CASE),
+}
 
 
 def parse_args(argv=None):
@@ -399,15 +413,15 @@ def run_ours(args, rank, world, local_rank):
     # DRAM traffic of the dominant kernel: ncu's dram bytes over the algorithmic bytes on a
     # small case of the same kernel and per-expert load, times this launch's algorithmic
     # bytes; None where no capture of the kernel as built stands
-    traffic_ratio = TRAFFIC_RATIO.get((args.workload, args.weights))
-    rl["traffic"] = traffic_ratio * wk["bytes_up"] if traffic_ratio is not None else None
-    rl["traffic_source"] = ("ncu dram bytes / algorithmic bytes = %.3f on the T=1024 E=2 case, "
-                            "times this launch's algorithmic bytes" % traffic_ratio
-                            if traffic_ratio is not None else None)
+    up_ratio = TRAFFIC_RATIO.get((args.workload, args.weights))
+    rl["traffic"] = up_ratio[0] * wk["bytes_up"] if up_ratio is not None else None
+    rl["traffic_source"] = ("ncu dram bytes / algorithmic bytes = %.3f on the %s, "
+                            "times this launch's algorithmic bytes" % up_ratio
+                            if up_ratio is not None else None)
     rl = {"kernel": KERNEL_NAMES[4], **rl}
     rl_down = kernel_roofline(wk["flops_down"], wk["bytes_down"], k_down, tensor_peak, hbm_peak)
     down_ratio = DOWN_TRAFFIC_RATIO.get((args.workload, args.weights))
-    rl_down["traffic"] = down_ratio * wk["bytes_down"] if down_ratio is not None else None
+    rl_down["traffic"] = down_ratio[0] * wk["bytes_down"] if down_ratio is not None else None
     roof_ms = max(wk["flops"] / (tensor_peak * 1e12),
                   (wk["w_bytes"] + wk["act_bytes"]) / (hbm_peak * 1e9)) * 1e3
     roof_ms_sust = max(wk["flops"] / (tensor_sust * 1e12),
