@@ -88,6 +88,10 @@ struct TcGroup {
   const float* b_scale0;
   const float* b_scale1;
   int64_t b_scale_stride;
+  // Routed groups of the swapped-operand kernel (tc_ws_gemm.cuh): assignments
+  // per expert and the capacity (-1: none), which give each tile's valid rows
+  const int32_t* counts;
+  int64_t cap;
 };
 
 struct TcParams {
