@@ -44,8 +44,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Algorithmic bytes are step_work's on the captured case (two experts).
 _PREFILL_CASE = "T=1024 E=2 case (1024 rows per expert)"
 _DECODE_CASE = "T=32 E=2 case"
+_DSV3_CASE = "T=1024 E=32 d=7168 d_e=2048 k=8 +shared case (256 rows per expert)"
 TRAFFIC_RATIO = {
-    ("mixtral", "dtype"): (538.84 / 545.26, _PREFILL_CASE),
+    ("mixtral", "dtype"): (538.90 / 545.26, _PREFILL_CASE),
+    ("deepseek_v3", "dtype"): (2196.70 / 2107.64, _DSV3_CASE),
     ("mixtral", "fp8"): (300.30 / 310.60, _PREFILL_CASE),
     ("decode", "fp8"): (240.30 / 237.46, _DECODE_CASE),
     ("decode", "mxfp4"): (131.30 / 127.43, _DECODE_CASE),
@@ -53,6 +55,7 @@ TRAFFIC_RATIO = {
 # the same for the down kernel
 DOWN_TRAFFIC_RATIO = {
     ("mixtral", "dtype"): (344.20 / 310.38, _PREFILL_CASE),
+    ("deepseek_v3", "dtype"): (1128.80 / 1138.75, _DSV3_CASE),
     ("mixtral", "fp8"): (220.10 / 192.97, _PREFILL_CASE),
     ("decode", "fp8"): (124.10 / 119.83, _DECODE_CASE),
     ("decode", "mxfp4"): (65.90 / 64.79, _DECODE_CASE),
@@ -68,7 +71,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="mixtral",
                     choices=["mixtral", "deepseek_v3", "switch_zipf", "decode", "tiny_fp32",
                              "mixtral_profile", "decode_profile", "routing_profile",
-                             "dsv3_routing_profile"])
+                             "dsv3_routing_profile", "dsv3_profile"])
     ap.add_argument("--weights", choices=["dtype", "fp8", "w8a8", "mxfp4"], default="dtype",
                     help="expert weights in the activation dtype; E4M3 codes with per-row "
                          "scales (quantised once by the library before timing); those and "
@@ -88,7 +91,7 @@ def workload_by_name(name):
             "decode": I.MIXTRAL_DECODE, "tiny_fp32": I.TINY_F32,
             "mixtral_profile": I.MIXTRAL_PROFILE, "decode_profile": I.DECODE_PROFILE,
             "routing_profile": I.ROUTING_PROFILE,
-            "dsv3_routing_profile": I.DSV3_ROUTING_PROFILE}[name]
+            "dsv3_routing_profile": I.DSV3_ROUTING_PROFILE, "dsv3_profile": I.DSV3_PROFILE}[name]
 
 
 def load_peaks():

@@ -83,6 +83,11 @@ DECODE_PROFILE = Workload("decode-shape-profile T=32 d=4096 E=2 d_e=14336 k=2",
 # experts, so the whole case holds about 0.2 GB, for hardware-counter captures.
 ROUTING_PROFILE = Workload("routing-kernels-profile T=4096 d=4096 E=8 d_e=256 k=2",
                            4096, 4096, 8, 256, 2, seed=1)
+# The DeepSeek-V3 expert shape (d = 7168, d_e = 2048, k = 8, the shared expert)
+# with 32 experts and 1024 tokens: the full layer's load of 256 routed rows per
+# expert, so the same kernel choices, with about 3 GB on the device.
+DSV3_PROFILE = Workload("dsv3-shape-profile T=1024 d=7168 E=32 d_e=2048 k=8 +shared 2048",
+                        1024, 7168, 32, 2048, 8, d_s=2048, seed=2)
 # The DeepSeek-V3-shaped router (T, d, E and k of that layer) with narrow
 # experts, about 1 GB on the device.
 DSV3_ROUTING_PROFILE = Workload("dsv3-routing-profile T=8192 d=7168 E=256 d_e=64 k=8",
