@@ -79,6 +79,9 @@ def parse_args(argv=None):
                          "per-32 block scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-streams", type=int, default=4,
+                    help="host threads (each with its own stream, workspace and buffers) "
+                         "taking alternate steps in the end-to-end timing")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode-shape leg of the default Mixtral-shaped run")
     ap.add_argument("--decode-calls", type=int, default=1000)
@@ -458,15 +461,15 @@ def run_ours(args, rank, world, local_rank):
     }
 
     # end to end through the host-buffer entry point: H2D x, forward, D2H y/aux/counts.
-    # moe_forward_host_io returns once its stream is done, so two host threads, each
-    # with its own stream, workspace and buffers, take alternate steps: one step's copies
-    # overlap the other's kernels, and every step still copies its own x in and its own
-    # y, aux and counts out inside the timed region.
+    # moe_forward_host_io returns once its stream is done, so several host threads (4 by
+    # default), each with its own stream, workspace and buffers, take turns: one step's
+    # copies overlap the others' kernels, and every step still copies its own x in and
+    # its own y, aux and counts out inside the timed region.
     if not args.no_e2e:
         import threading
         ke = min(args.steps, 100)
-        NSTR = 2
-        streams = [stream, torch.cuda.Stream(dev)]
+        NSTR = args.e2e_streams
+        streams = [stream] + [torch.cuda.Stream(dev) for _ in range(NSTR - 1)]
         x_host = [xs[j].cpu().pin_memory() for j in range(2)]
         nbytes = ws.buf.numel()
         fmt = (_lib.MOE_WEIGHTS_FP8_W8A8 if act_fp8 else
@@ -510,11 +513,13 @@ def run_ours(args, rank, world, local_rank):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(streams[0])
-        streams[1].wait_event(e0)
+        for sx in streams[1:]:
+            sx.wait_event(e0)
         e2e_steps(0, ke)
-        done1 = torch.cuda.Event()
-        done1.record(streams[1])
-        streams[0].wait_event(done1)
+        for sx in streams[1:]:
+            done = torch.cuda.Event()
+            done.record(sx)
+            streams[0].wait_event(done)
         e1.record(streams[0])
         torch.cuda.synchronize()
         barrier()
