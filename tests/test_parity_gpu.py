@@ -32,8 +32,13 @@ SMALL = [
     Workload("bf16 shared+capacity", 700, 256, 8, 256, 2, d_s=256, capacity_factor=0.8, seed=21),
     Workload("fp32 shared+capacity", 333, 128, 8, 96, 2, "f32", d_s=64, capacity_factor=0.7, seed=22),
     Workload("fp32 ragged", 257, 96, 5, 160, 3, "f32", seed=23),
-    # >= 512 routed rows per expert run the down GEMM on CTA pairs (cta_group::2),
-    # >= 2048 the gate/up GEMM as well
+    # more than 64 tokens and up to 2048 (gate/up) or 512 (down) routed rows per
+    # expert: the swapped-operand kernels, token tiles sized to their valid rows
+    Workload("bf16 T=65, smallest swapped batch", 65, 256, 8, 256, 2, seed=35),
+    Workload("bf16 about 3 rows per expert (N=16 tiles), shared", 100, 256, 64, 128, 2, d_s=64,
+             seed=36),
+    # > 512 routed rows per expert run the down GEMM on CTA pairs (cta_group::2),
+    # > 2048 the gate/up GEMM as well
     Workload("pair odd tile counts", 4300, 256, 2, 320, 1, seed=24),
     Workload("pair shared expert", 4200, 256, 2, 256, 1, d_s=128, seed=25),
     Workload("pair both GEMMs k=2", 2200, 256, 2, 192, 2, seed=28),
