@@ -126,11 +126,23 @@ __global__ void __launch_bounds__(256) combine_kernel(
     float acc[VN];
 #pragma unroll
     for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-    for (int s = 0; s < k; ++s) {
-      const int p = __shfl_sync(0xffffffffu, mypos, s);
-      if (p >= 0 && active) {
+    // four slots' loads in flight at once (separate registers), then summed in
+    // slot order, so the result is the same as one slot at a time
+    for (int s0 = 0; s0 < k; s0 += 4) {
+      uint4 v[4];
+      bool has[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = s0 + j;
+        const int p = __shfl_sync(0xffffffffu, mypos, s < k ? s : 0);
+        has[j] = s < k && p >= 0 && active;
+        if (has[j]) v[j] = ld_v4(reinterpret_cast<const uint4*>(yrows + (size_t)p * d) + c);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!has[j]) continue;
         float f[VN];
-        Vec16<TY>::unpack(ld_v4(reinterpret_cast<const uint4*>(yrows + (size_t)p * d) + c), f);
+        Vec16<TY>::unpack(v[j], f);
 #pragma unroll
         for (int i = 0; i < VN; ++i) acc[i] += f[i];
       }
