@@ -253,18 +253,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // broadcast by shuffle (a load per element would wait once per store)
           const float rs = (g.row_scale != nullptr && c0 + lane < v)
                                ? g.row_scale[ti.row0 + c0 + lane] : 1.f;
-          float sc[32];
+          const int col0 = ti.nb * 2 * BM + r, col1 = col0 + BM;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) sc[c] = __shfl_sync(0xffffffffu, rs, c);
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm) {
-            const int col = ti.nb * 2 * BM + mm * BM + r;
-            if (col < g.N) {
-              const float* dv = mm == 0 ? d0 : d1;
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c0 + c < v)
-                  out[(size_t)(ti.row0 + c0 + c) * g.N + col] = __float2bfloat16_rn(sc[c] * dv[c]);
+          for (int c = 0; c < 32; ++c) {
+            const float sc = __shfl_sync(0xffffffffu, rs, c);  // warp-uniform point
+            if (c0 + c < v) {
+              __nv_bfloat16* o = out + (size_t)(ti.row0 + c0 + c) * g.N;
+              if (col0 < g.N) o[col0] = __float2bfloat16_rn(sc * d0[c]);
+              if (col1 < g.N) o[col1] = __float2bfloat16_rn(sc * d1[c]);
             }
           }
         }
