@@ -46,8 +46,8 @@ _PREFILL_CASE = "T=1024 E=2 case (1024 rows per expert)"
 _DECODE_CASE = "T=32 E=2 case"
 _DSV3_CASE = "T=1024 E=32 d=7168 d_e=2048 k=8 +shared case (256 rows per expert)"
 TRAFFIC_RATIO = {
-    ("mixtral", "dtype"): (538.90 / 545.26, _PREFILL_CASE),
-    ("deepseek_v3", "dtype"): (2196.70 / 2107.64, _DSV3_CASE),
+    ("mixtral", "dtype"): (539.20 / 545.26, _PREFILL_CASE),
+    ("deepseek_v3", "dtype"): (2199.70 / 2107.64, _DSV3_CASE),
     ("mixtral", "fp8"): (300.30 / 310.60, _PREFILL_CASE),
     ("decode", "fp8"): (240.30 / 237.46, _DECODE_CASE),
     ("decode", "mxfp4"): (131.30 / 127.43, _DECODE_CASE),
@@ -55,7 +55,7 @@ TRAFFIC_RATIO = {
 # the same for the down kernel
 DOWN_TRAFFIC_RATIO = {
     ("mixtral", "dtype"): (344.20 / 310.38, _PREFILL_CASE),
-    ("deepseek_v3", "dtype"): (1128.80 / 1138.75, _DSV3_CASE),
+    ("deepseek_v3", "dtype"): (1129.70 / 1138.75, _DSV3_CASE),
     ("mixtral", "fp8"): (220.10 / 192.97, _PREFILL_CASE),
     ("decode", "fp8"): (124.10 / 119.83, _DECODE_CASE),
     ("decode", "mxfp4"): (65.90 / 64.79, _DECODE_CASE),
