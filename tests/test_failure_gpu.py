@@ -24,6 +24,7 @@ def _cuda():
     Workload("timeout routed", 1000, 512, 4, 320, 2, seed=41),
     Workload("timeout shared", 300, 256, 16, 128, 4, d_s=192, seed=42),
     Workload("timeout pair kernels", 4200, 256, 2, 256, 1, d_s=128, seed=43),
+    Workload("timeout token-major 32-row box", 20, 256, 4, 256, 2, seed=47),
 ], ids=lambda w: w.name)
 def test_expired_waits_are_reported_and_the_context_survives(w):
     inp = make_inputs(w, device="cuda")
