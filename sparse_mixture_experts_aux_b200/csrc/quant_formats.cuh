@@ -56,9 +56,13 @@ __device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t* o) {
 }
 
 // The fp16 multiplier 2^(X - 127) / row_factor of one MXFP4 block: a power of
-// two when the row factor is one (2^X_row), exact in fp16 down to 2^-24.
+// two when the row factor is one (2^X_row), exact in fp16 down to 2^-24. For
+// exponent codes 1..254, 2^(X - 127) is a normal fp32 built from its bits, and
+// one multiply gives the correctly rounded product, the value ldexpf returns;
+// codes 0 and 255 take ldexpf itself.
 __device__ __forceinline__ uint32_t mx_block_multiplier(uint32_t e8m0, float inv_row_factor) {
-  const float m = ldexpf(inv_row_factor, (int)e8m0 - 127);
+  const float m = (e8m0 - 1u < 254u) ? __uint_as_float(e8m0 << 23) * inv_row_factor
+                                     : ldexpf(inv_row_factor, (int)e8m0 - 127);
   const __half2 h = __float2half2_rn(m);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
