@@ -30,6 +30,8 @@ constexpr unsigned long long kDrainTimeoutNs = 2000000000ull;  // teardown waits
 // expert (T k / E) run the swapped-operand GEMMs (tc_ws_gemm.cuh)
 constexpr int64_t kWsUpMaxRowsPerExpert = 2048;   // gate/up
 constexpr int64_t kWsDownMaxRowsPerExpert = 512;  // down
+// above that, the down GEMM runs on CTA pairs, with the operands swapped
+constexpr bool kPairDownSwap = true;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -285,9 +287,9 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
   return cfg;
 }
 
-template <int EPI>
+template <int EPI, bool SWAP = false>
 bool pair_setup(int num_sms, int* clusters) {
-  auto kern = moe::tc2::tc2_grouped_gemm_kernel<EPI>;
+  auto kern = moe::tc2::tc2_grouped_gemm_kernel<EPI, SWAP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            moe::tc2::SMEM_BYTES) != cudaSuccess)
     return false;
@@ -337,8 +339,11 @@ moe_status device_setup(int* num_sms, int* pair_clusters = nullptr) {
         !wq_attr<moe::tc::EPI_SWIGLU_TC, moe::tcf8::WQ_MXFP4>() ||
         !wq_attr<moe::tc::EPI_SCALE_TC, moe::tcf8::WQ_MXFP4>())
       return MOE_ERR_CUDA;
+    int swap_clusters = 0;
     if (!pair_setup<moe::tc::EPI_SWIGLU_TC>(di.num_sms, &di.pair_clusters[0]) ||
-        !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]))
+        !pair_setup<moe::tc::EPI_SCALE_TC>(di.num_sms, &di.pair_clusters[1]) ||
+        !pair_setup<moe::tc::EPI_SCALE_TC, true>(di.num_sms, &swap_clusters) ||
+        swap_clusters != di.pair_clusters[1])
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(moe::rtc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              moe::rtc::SMEM_LIMIT) != cudaSuccess)
@@ -869,11 +874,18 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
       const int abox = pair_down ? moe::tc::BM : arows;
       moe::tc::TcMaps dn;
       memset(&dn, 0, sizeof(dn));
-      bool ok = encode_map(&dn.a[0], h, P.de, P.rows_max, 1, abox, 2) &&
-                encode_map(&dn.b0[0], W_d, P.de, P.d, E, brows, 3);
+      // swapped pairs: the weight map is A and the rows' map B
+      const bool swap = pair_down && kPairDownSwap;
+      const void* dn_rows[2] = {h, hs};
+      bool ok = swap ? encode_map(&dn.a[0], W_d, P.de, P.d, E, HB, 3) &&
+                           encode_map(&dn.b0[0], h, P.de, P.rows_max, 1, HB, 2)
+                     : encode_map(&dn.a[0], h, P.de, P.rows_max, 1, abox, 2) &&
+                           encode_map(&dn.b0[0], W_d, P.de, P.d, E, brows, 3);
       if (P.ds)
-        ok = ok && encode_map(&dn.a[1], hs, P.ds, P.T, 1, abox, 2) &&
-             encode_map(&dn.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, brows, 3);
+        ok = ok && (swap ? encode_map(&dn.a[1], sg + 2 * sh_n, P.ds, P.d, 1, HB, 3) &&
+                               encode_map(&dn.b0[1], dn_rows[1], P.ds, P.T, 1, HB, 2)
+                         : encode_map(&dn.a[1], hs, P.ds, P.T, 1, abox, 2) &&
+                               encode_map(&dn.b0[1], sg + 2 * sh_n, P.ds, P.d, 1, brows, 3));
       if (!ok) return MOE_ERR_CUDA;
       dn.b1[0] = dn.b0[0];
       dn.b1[1] = dn.b0[1];
@@ -886,13 +898,18 @@ moe_status forward_impl(const moe_dims* dims, const void* x, const float* W_r, c
         td.call_err = call_err;
         td.g[0] = {tile_start, pair_start, E, rows_cap, (P.d + BNp - 1) / BNp, P.de / moe::tc::BK, P.d,
                    yrows, rowgate};
+        td.g[0].counts = counts;
+        td.g[0].cap = P.C;
         if (P.ds)
           td.g[1] = {nullptr, nullptr, 1, T, (P.d + BNp - 1) / BNp, P.ds / moe::tc::BK, P.d, ys,
                      nullptr};
         cudaLaunchConfig_t cfg = pair_config<moe::tc::EPI_SCALE_TC>(pair_clusters[1], st, attr, true);
-        if (cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
-                               dn, td) != cudaSuccess)
-          return MOE_ERR_CUDA;
+        const cudaError_t le =
+            swap ? cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC, true>,
+                                      dn, td)
+                 : cudaLaunchKernelEx(&cfg, moe::tc2::tc2_grouped_gemm_kernel<moe::tc::EPI_SCALE_TC>,
+                                      dn, td);
+        if (le != cudaSuccess) return MOE_ERR_CUDA;
       } else {
         moe::tc::TcParams tp{};
         tp.num_groups = ng;

@@ -60,6 +60,10 @@ struct Tc2Group {
   int N;                      // output columns
   void* out;                  // bf16 [rows, N]
   const float* row_scale;     // scale epilogue: factor per row; NULL = 1
+  // SWAP kernels: assignments per expert and the capacity (-1: none), which
+  // give each token tile's valid rows
+  const int32_t* counts;
+  int64_t cap;
 };
 
 struct Tc2Params {
@@ -243,9 +247,33 @@ __device__ __forceinline__ bool pair_out_of_bounds(const PairTile& t, const Tc2G
 #endif
 }
 
-template <int EPI>
+// SWAP kernels: valid token rows of a pair tile's 256-row token tile, 1..256
+// (routed groups: the expert's kept rows past the tile's start; dense: the
+// group's rows).
+__device__ __forceinline__ int pair_rows(const PairTile& t, const Tc2Group& g,
+                                         const int32_t* s_ts) {
+  int v;
+  if (t.g == 0 && g.tile_start != nullptr) {
+    int kept = g.counts[t.e];
+    if (g.cap >= 0 && kept > g.cap) kept = static_cast<int>(g.cap);
+    v = kept - (t.row0 - s_ts[t.e] * HALF_M);
+  } else {
+    v = g.rows - t.row0;
+  }
+  return v < 1 ? 1 : (v > 2 * HALF_M ? 2 * HALF_M : v);
+}
+
+// SWAP (down GEMM only): the operands swapped, as in tc_ws_gemm.cuh. A = 256
+// rows of W_d across the pair (128 per CTA: maps.a is the weight map), B = the
+// tile's 256-row token tile (maps.b0, the rows' map): each CTA loads its half,
+// N / 2 rows from row0 + (N / 2) rank, N = the tile's valid rows rounded up to
+// 16, so the segment padding of an expert's last tile is not multiplied. Each
+// CTA's TMEM holds its 128 weight rows x N tokens; the epilogue stores
+// transposed (lane = output column).
+template <int EPI, bool SWAP = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ TcMaps maps, const Tc2Params p) {
+  static_assert(!SWAP || EPI == tc::EPI_SCALE_TC, "swapped operands: the down GEMM");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = tc::smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -333,6 +361,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const int kbs = p.g[ti.g].k_blocks;
         const int arow = ti.row0 + HALF_M * (int)rank;
+        // SWAP: this CTA's half of the token tile starts N / 2 rows in for the peer
+        const int brow = SWAP ? ti.row0 + ((pair_rows(ti, p.g[ti.g], s_ts) + 15) & ~15) / 2 *
+                                              (int)rank
+                              : 0;
         for (int kb = 0; kb < kbs; ++kb) {
           if (!wait_pair_fast(empty_bar(stage), phase ^ 1u, abort_flag, peer_abort, tmo)) {
             ok = false;
@@ -342,11 +374,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb_leader = mapa_shared(full_bar(stage), 0u);
           if (leader) tc::mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          tma_load_2d_pair(sa, &maps.a[ti.g], fb_leader, kb * BK, arow);
-          if (EPI == tc::EPI_SWIGLU_TC) {
+          if constexpr (SWAP) {
+            tma_load_3d_pair(sa, &maps.a[ti.g], fb_leader, kb * BK, ti.nb * BN + 128 * (int)rank,
+                             ti.e);
+            tma_load_2d_pair(sb, &maps.b0[ti.g], fb_leader, kb * BK, brow);
+          } else if (EPI == tc::EPI_SWIGLU_TC) {
+            tma_load_2d_pair(sa, &maps.a[ti.g], fb_leader, kb * BK, arow);
             tma_load_3d_pair(sb, leader ? &maps.b0[ti.g] : &maps.b1[ti.g], fb_leader, kb * BK,
                              ti.nb * (BN / 2), ti.e);
           } else {
+            tma_load_2d_pair(sa, &maps.a[ti.g], fb_leader, kb * BK, arow);
             tma_load_3d_pair(sb, &maps.b0[ti.g], fb_leader, kb * BK,
                              ti.nb * BN + 128 * (int)rank, ti.e);
           }
@@ -374,6 +411,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const PairTile ti = decode_pair(tile, tiles0, p, s_ts, s_ps);
         if (pair_out_of_bounds(ti, p.g[ti.g])) continue;
         const int kbs = p.g[ti.g].k_blocks;
+        const uint32_t idesc =
+            SWAP ? tc::make_idesc(2 * HALF_M, (pair_rows(ti, p.g[ti.g], s_ts) + 15) & ~15) : IDESC;
         if (!wait_pair(tempty_bar(acc), acc_phase ^ 1u, abort_flag, peer_abort, tmo)) {
           ok = false;
           break;
@@ -391,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t bd = tc::sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -423,6 +462,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc::tc_fence_after();
+      if constexpr (SWAP) {
+        // lane = this CTA's weight row (output column), columns = the tile's tokens
+        const int v = pair_rows(ti, g, s_ts);
+        const int col = ti.nb * BN + 128 * (int)rank + r_in_half;
+        const uint32_t tb = tmem_base + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out);
+#pragma unroll 1
+        for (int c = half; c * 32 < v; c += 2) {
+          float d[32];
+          __syncwarp();
+          tc::tmem_ld32(tb + c * 32, d);
+          const int c0 = c * 32;
+          // the 32 tokens' gate scales: one load, broadcast at a warp-uniform point
+          const float rs = (g.row_scale != nullptr && c0 + lane < v)
+                               ? g.row_scale[ti.row0 + c0 + lane] : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            const float sc = __shfl_sync(0xffffffffu, rs, cc);
+            if (c0 + cc < v && col < g.N)
+              out[(size_t)(ti.row0 + c0 + cc) * g.N + col] = __float2bfloat16_rn(sc * d[cc]);
+          }
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0u));
+        acc ^= 1u;
+        if (acc == 0u) acc_phase ^= 1u;
+        continue;
+      }
       const int row = ti.row0 + HALF_M * (int)rank + r_in_half;
       const bool row_ok =
           ti.half_valid[rank] && ((g.tile_start != nullptr) || row < g.rows);
