@@ -54,7 +54,7 @@ TRAFFIC_RATIO = {
 }
 # the same for the down kernel
 DOWN_TRAFFIC_RATIO = {
-    ("mixtral", "dtype"): (344.20 / 310.38, _PREFILL_CASE),
+    ("mixtral", "dtype"): (343.40 / 310.38, _PREFILL_CASE),
     ("deepseek_v3", "dtype"): (1129.70 / 1138.75, _DSV3_CASE),
     ("mixtral", "fp8"): (220.10 / 192.97, _PREFILL_CASE),
     ("decode", "fp8"): (124.10 / 119.83, _DECODE_CASE),
