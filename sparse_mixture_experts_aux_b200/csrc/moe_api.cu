@@ -530,7 +530,7 @@ moe_status launch_route_and_permute(const Plan& P, const moe_dims* dims, const T
   // (2) scan: counts, capacity, segment offsets, aux
   tm.at(4);
   if (!fused_scan)
-    launch_pdl(moe::scan_kernel, 1, moe::scan_threads(P.E), 0, st, hist, P.nblk, psum_part, P.nblk, P.E, P.T, P.k, P.C, counts, base, tile_start, pair_start,
+    launch_pdl(moe::scan_kernel, 1, moe::scan_kernel_threads(P.E), 0, st, hist, P.nblk, psum_part, P.nblk, P.E, P.T, P.k, P.C, counts, base, tile_start, pair_start,
         probsum, aux, sa.call_err, P.rows_max);
   tm.at(5);
   if (launched() != MOE_OK) return MOE_ERR_CUDA;

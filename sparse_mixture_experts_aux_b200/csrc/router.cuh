@@ -459,24 +459,67 @@ __device__ void scan_experts(int nthreads, const int32_t* __restrict__ hist, int
                              int32_t* __restrict__ base, int32_t* __restrict__ tile_start,
                              int32_t* __restrict__ pair_start, double* __restrict__ probsum,
                              float* __restrict__ aux, int* __restrict__ call_err, int64_t rows_max,
-                             int* s_scan, double* s_sum) {
+                             int* s_scan, double* s_sum, int* s_cnt = nullptr,
+                             double* s_psd = nullptr) {
   const int e = threadIdx.x;
   if (e == 0 && call_err != nullptr) *call_err = 0;  // the GEMMs of this call run after this
+  if (s_cnt != nullptr) {
+    // A warp per expert: each lane takes a contiguous range of chunks, a shuffle
+    // scan turns the range sums into each range's start, and the lanes write the
+    // chunks' bases; the probability partials are loaded 32 at a time and added
+    // in part order, as one thread would.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int per = (nblk + 31) / 32;
+    for (int ee = warp; ee < E; ee += nw) {
+      const int b0 = lane * per < nblk ? lane * per : nblk;
+      const int b1 = b0 + per < nblk ? b0 + per : nblk;
+      int local = 0;
+      for (int b = b0; b < b1; ++b) local += hist[(size_t)b * E + ee];
+      int incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      int run = incl - local;
+      for (int b = b0; b < b1; ++b) {
+        base[(size_t)b * E + ee] = run;
+        run += hist[(size_t)b * E + ee];
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      double ps = 0.0;
+      for (int p0 = 0; p0 < nparts; p0 += 32) {
+        const double v = p0 + lane < nparts ? psum_part[(size_t)(p0 + lane) * E + ee] : 0.0;
+        const int n = nparts - p0 < 32 ? nparts - p0 : 32;
+        for (int j = 0; j < n; ++j) ps += __shfl_sync(0xffffffffu, v, j);
+      }
+      if (lane == 0) {
+        s_cnt[ee] = total;
+        s_psd[ee] = ps;
+      }
+    }
+    __syncthreads();
+  }
   int tiles = 0;
   double term = 0.0;
   if (e < E) {
     int run = 0;
+    double ps = 0.0;
+    if (s_cnt != nullptr) {
+      run = s_cnt[e];
+      ps = s_psd[e];
+    } else {
 #pragma unroll 8
-    for (int b = 0; b < nblk; ++b) {
-      base[(size_t)b * E + e] = run;
-      run += hist[(size_t)b * E + e];
+      for (int b = 0; b < nblk; ++b) {
+        base[(size_t)b * E + e] = run;
+        run += hist[(size_t)b * E + e];
+      }
+#pragma unroll 8
+      for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
     }
     counts[e] = run;
     const int kept = (C >= 0 && (int64_t)run > C) ? (int)C : run;
     tiles = (kept + ROW_TILE - 1) / ROW_TILE;
-    double ps = 0.0;
-#pragma unroll 8
-    for (int p = 0; p < nparts; ++p) ps += psum_part[(size_t)p * E + e];
     probsum[e] = ps;
     term = (double)run * ps;
   }
@@ -534,6 +577,14 @@ __host__ __device__ inline int scan_threads(int E) {
   int n = 32;
   while (n < E) n <<= 1;
   return n;
+}
+// Threads of the scan kernel. Up to 32 experts: a warp per expert (at least 8
+// warps) walks the expert's chunks in parallel; above that a thread per expert
+// walks them in sequence, as many experts at once.
+constexpr int SCAN_WARP_PATH_MAX_E = 32;
+__host__ __device__ inline int scan_kernel_threads(int E) {
+  if (E <= SCAN_WARP_PATH_MAX_E) return 32 * E < 256 ? 256 : 32 * E;
+  return scan_threads(E);
 }
 
 // Arguments of the scan when the routing kernel runs it itself (one chunk).
@@ -802,8 +853,7 @@ __global__ void __launch_bounds__(256, 1) route_kernel(
   }
 }
 
-// The scan as its own kernel: one block of nthreads = the smallest power of two
-// >= max(E, 32) threads.
+// The scan as its own kernel: one block of scan_kernel_threads(E) threads.
 __global__ void __launch_bounds__(1024) scan_kernel(
     const int32_t* __restrict__ hist, int nblk, const double* __restrict__ psum_part, int nparts,
     int E, int64_t T, int k, int64_t C, int32_t* __restrict__ counts, int32_t* __restrict__ base,
@@ -814,8 +864,12 @@ __global__ void __launch_bounds__(1024) scan_kernel(
   pdl_launch_dependents();
   __shared__ int s_scan[2 * 1024];
   __shared__ double s_sum[1024];
+  __shared__ int s_cnt[1024];
+  __shared__ double s_psd[1024];
+  const bool warp_path = E <= SCAN_WARP_PATH_MAX_E;
   scan_experts(blockDim.x, hist, nblk, psum_part, nparts, E, T, k, C, counts, base, tile_start,
-               pair_start, probsum, aux, call_err, rows_max, s_scan, s_sum);
+               pair_start, probsum, aux, call_err, rows_max, s_scan, s_sum,
+               warp_path ? s_cnt : nullptr, warp_path ? s_psd : nullptr);
 }
 
 
