@@ -21,6 +21,9 @@
 // Rows are grouped per expert in 128-row segments; a pair tile covers two
 // consecutive 128-row tiles of one expert, and when an expert has an odd tile
 // count the peer half of its last pair is computed but not stored.
+// The SWAP form (down GEMM) exchanges the roles: A is 256 weight rows across
+// the pair and B the pair tile's token rows, with N set per tile to its valid
+// rows rounded up to 16, so the odd expert's last tile is not padded.
 #pragma once
 #include "tc_gemm.cuh"
 
